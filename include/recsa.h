@@ -1,0 +1,197 @@
+/*
+ * recsa.h - C ABI of the RecSA (Recursive Sparse Attention) tree build and
+ * level-wise sparse attend for NVIDIA B200 (sm_100a).
+ *
+ * Method: "Recursive Sparse Attention: Million-Token Length Extrapolation at
+ * Logarithmic Cost" (arXiv 2611.07232), abstract.  A tree is built over the KV
+ * cache; every node summarises its subtree with one key (a per-layer pooler that
+ * all levels share) and one mean-pooled value.  A query descends the tree one
+ * level at a time, keeping at most k candidates per level above the tokens; the
+ * summaries of the candidates it does not keep share one softmax with the exact
+ * tokens under the kept leaves, and every entry is RoPE-rotated at its index among
+ * the candidates of its level.
+ *
+ * Readings this library implements where the abstract is silent:
+ *   - pooler: parent key = W @ (mean of the children's stored pre-RoPE keys), W a
+ *     caller-supplied fp32 128x128 row-major matrix, applied at every level;
+ *   - parent value = token-count-weighted mean of the children's values (= mean of
+ *     the subtree's tokens); node rows are stored as bf16 (round to nearest even);
+ *   - levels: n_0 = L, n_{l+1} = ceil(n_l / b) while n_l > b (the top level has at
+ *     most b nodes; L <= b means plain attention over the tokens);
+ *   - selection ranks candidates by the sum, over the query heads of a KV group
+ *     (heads g*G .. g*G+G-1), of the scaled logits; ties go to the lower node index;
+ *   - the RoPE position of a candidate is its rank among its level's candidates in
+ *     node order and the query's position is that level's candidate count;
+ *     rotate-half RoPE over dims (i, i+64), angle pos * base^(-2i/128);
+ *   - a query at position p sees tokens [0, p): decode queries sit at p = L; query i
+ *     of a prefill chunk appended at L sits at p = L + i.  In prefill the partial
+ *     trailing node of each level is not scored, takes no top-k slot, holds a
+ *     position and is always expanded;
+ *   - a query with nothing visible (prefill query 0 of an empty cache) outputs zeros.
+ *
+ * Conventions for every call:
+ *   - data pointers are DEVICE pointers (CUDA global memory of the current device)
+ *     unless stated; bf16 tensors are IEEE bfloat16, contiguous, row-major, and
+ *     every base pointer must be 16-byte aligned;
+ *   - the caller owns every buffer and keeps it alive until the work queued on
+ *     `stream` has finished; no call allocates or frees device memory;
+ *   - calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and never synchronise, except recsa_check_device_errors;
+ *   - argument errors are reported synchronously with a status and nothing is
+ *     launched; a failed launch returns RECSA_ERR_CUDA; recsa_last_error() gives a
+ *     thread-local description of the most recent failure;
+ *   - the library holds no device state of its own; calls on different streams
+ *     with disjoint outputs may run concurrently.
+ */
+#ifndef RECSA_H
+#define RECSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(_WIN32)
+#define RECSA_API
+#else
+#define RECSA_API __attribute__((visibility("default")))
+#endif
+
+typedef struct CUstream_st *recsa_stream_t; /* ABI-identical to cudaStream_t */
+
+typedef enum recsa_status {
+  RECSA_OK = 0,
+  RECSA_ERR_INVALID_ARGUMENT = 1,    /* null/misaligned pointer, bad size or shape  */
+  RECSA_ERR_UNSUPPORTED = 2,         /* valid but outside what the kernels handle   */
+  RECSA_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes below recsa_workspace_size()       */
+  RECSA_ERR_CAPACITY = 4,            /* length + chunk exceeds the cache capacity   */
+  RECSA_ERR_CUDA = 5,                /* a CUDA runtime call or launch failed        */
+  RECSA_ERR_DEVICE_CHECK = 6,        /* a kernel found an out-of-range index or a
+                                        workspace that was not initialised          */
+  RECSA_ERR_TIMEOUT = 7              /* a bounded device-side wait ran out          */
+} recsa_status;
+
+#define RECSA_HEAD_DIM 128
+#define RECSA_TOPK_ALL 0x7fffffff /* keep every candidate (full expansion) */
+#define RECSA_MAX_LEVELS 40       /* levels above the tokens a tree may have */
+#define RECSA_MAX_CANDIDATES 4096 /* per level and query group (see recsa_decode) */
+
+/* Per-layer attention shape and method parameters. */
+typedef struct recsa_params {
+  int32_t head_dim;     /* must be 128                                              */
+  int32_t num_kv_heads; /* Hkv >= 1                                                 */
+  int32_t num_q_heads;  /* Hq = G * Hkv with G (query heads per KV group) 1, 2, 4, 8 */
+  int32_t branching;    /* b >= 2 children per node                                 */
+  int32_t top_k;        /* k >= 0 kept per level above the tokens, or RECSA_TOPK_ALL */
+  float rope_base;      /* > 0, e.g. 1e6                                            */
+  float softmax_scale;  /* > 0, or 0 for 1/sqrt(128)                                */
+} recsa_params;
+
+/* One layer's KV cache and its summary tree.
+ *   k_tok, v_tok : bf16 [batch][Hkv][capacity][128], pre-RoPE token keys / values;
+ *                  slots [0, length) are valid.
+ *   k_node, v_node: bf16 node arena, each [node_rows][128] with the layout that
+ *                  recsa_tree_layout() returns for (batch, capacity); level l,
+ *                  sequence s, KV head h, node j sits at row
+ *                  level_row_offsets[l] + (s*Hkv + h) * ceil(capacity / b^l) + j.
+ *   pooler       : fp32 [128][128] row-major W (node key = W @ mean of child keys).
+ * All sequences share `length`. */
+typedef struct recsa_tree {
+  int32_t batch;
+  int32_t reserved;
+  int64_t capacity;
+  int64_t length;
+  void *k_tok;
+  void *v_tok;
+  void *k_node;
+  void *v_node;
+  const float *pooler;
+} recsa_tree;
+
+/* Optional diagnostics of recsa_decode / recsa_prefill_chunk (pass NULL for none).
+ * A "tile" is one (sequence, query, KV group); tiles are numbered
+ * ((s * Hkv + g) * num_queries + query).
+ *   sel_idx  : int32 [tiles][sel_levels][top_k]; slot (l-1) receives the node indices
+ *              kept at level l (ascending, -1 padded).  Needs top_k <= 64.
+ *   entries  : int32 [tiles][2]; keys scored and values folded by the tile (rows read).
+ *   cluster_size: 0 = automatic; 1, 2 or 4 forces the number of CTAs that share one
+ *              tile (a launch-shape choice; results are identical up to rounding). */
+typedef struct recsa_debug {
+  int32_t *sel_idx;
+  int32_t sel_levels;
+  int32_t cluster_size;
+  int32_t *entries;
+} recsa_debug;
+
+/* Arena layout of a tree of `capacity` token slots (host only, no CUDA call).
+ * Writes the total node rows (per K and per V arena), the number of levels above
+ * the tokens for a cache filled to capacity, and level_row_offsets[0..levels]
+ * (entry 0 is 0 and unused).  The arena size in bytes is node_rows * 256. */
+RECSA_API recsa_status recsa_tree_layout(const recsa_params *params, int32_t batch, int64_t capacity,
+                                         int64_t *node_rows_out, int32_t *num_levels_out,
+                                         int64_t level_row_offsets_out[RECSA_MAX_LEVELS + 1]);
+
+/* Bytes of the workspace that recsa_decode / recsa_prefill_chunk need for trees of
+ * up to `capacity` tokens with these params (host only).  The workspace holds the
+ * RoPE cos/sin table and the device error word. */
+RECSA_API recsa_status recsa_workspace_size(const recsa_params *params, int64_t capacity, size_t *bytes_out);
+
+/* Fill a workspace of ws_bytes >= recsa_workspace_size(params, capacity) bytes
+ * (device pointer, 16-byte aligned): computes the RoPE table in fp64 and clears the
+ * error word.  Call once per (params, capacity) before the first attend call that
+ * uses this workspace; its contents then stay valid for every later call. */
+RECSA_API recsa_status recsa_workspace_init(const recsa_params *params, int64_t capacity, void *ws,
+                                            size_t ws_bytes, recsa_stream_t stream);
+
+/* Build every level of the tree over the first tree->length tokens (abstract: each
+ * node summarises its subtree with one pooled key and one mean-pooled value).
+ * Overwrites the node arena rows of levels 1..T(length). */
+RECSA_API recsa_status recsa_build_tree(const recsa_params *params, const recsa_tree *tree,
+                                        recsa_stream_t stream);
+
+/* Decode attention of num_queries independent queries per sequence, all at position
+ * L = tree->length, over a tree built by recsa_build_tree (abstract: level-wise
+ * selection of at most k candidates, unselected summaries sharing one softmax with
+ * the exact tokens).
+ *   q   : bf16 [batch][num_queries][Hq][128], pre-RoPE.
+ *   out : [batch][num_queries][Hq][128], fp32 if out_is_fp32 else bf16.
+ *   ws  : an initialised workspace (recsa_workspace_init) for >= tree->capacity.
+ * Needs length >= 1 and at most RECSA_MAX_CANDIDATES candidates per level
+ * (max(b, min(k*b, L)) here), else RECSA_ERR_UNSUPPORTED. */
+RECSA_API recsa_status recsa_decode(const recsa_params *params, const recsa_tree *tree, const void *q,
+                                    int32_t num_queries, void *out, int32_t out_is_fp32, void *ws,
+                                    size_t ws_bytes, const recsa_debug *debug, recsa_stream_t stream);
+
+/* Causal prefill of a chunk of `chunk` tokens at positions L .. L+chunk-1
+ * (L = tree->length): appends k_new / v_new to the token caches, rebuilds the tree
+ * nodes those tokens touch (and any level that becomes new), then attends query i
+ * at p = L + i.  On success tree->length becomes L + chunk (host-side update; the
+ * device work is still queued).
+ *   k_new, v_new: bf16 [batch][chunk][Hkv][128]; q: bf16 [batch][chunk][Hq][128];
+ *   out: [batch][chunk][Hq][128] (fp32 or bf16).
+ * Needs L + chunk <= capacity (else RECSA_ERR_CAPACITY) and at most
+ * RECSA_MAX_CANDIDATES candidates per level (max(b, min((k+1)*b, L+chunk))). */
+RECSA_API recsa_status recsa_prefill_chunk(const recsa_params *params, recsa_tree *tree, const void *k_new,
+                                           const void *v_new, const void *q, int32_t chunk, void *out,
+                                           int32_t out_is_fp32, void *ws, size_t ws_bytes,
+                                           const recsa_debug *debug, recsa_stream_t stream);
+
+/* Synchronise `stream`, then read and clear the workspace's device error word.
+ * Returns RECSA_OK, RECSA_ERR_DEVICE_CHECK (an index out of range, or a workspace
+ * that was not initialised for the call), RECSA_ERR_TIMEOUT (a bounded wait ran
+ * out), or RECSA_ERR_CUDA. */
+RECSA_API recsa_status recsa_check_device_errors(void *ws, recsa_stream_t stream);
+
+/* Static name of a status code. */
+RECSA_API const char *recsa_status_string(recsa_status status);
+
+/* Thread-local description of the most recent failure in this thread ("" if none). */
+RECSA_API const char *recsa_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RECSA_H */
