@@ -1,0 +1,551 @@
+"""Benchmark of the RecSA hot path on B200 (one JSON line on stdout).
+
+Headline: decode queries/s at a 1M-token context (B = 4 sequences, 32 query / 8 KV
+heads, head_dim 128, b = 16, k = 8, one query per sequence), each step one
+recsa_decode call over a tree built beforehand, L2 flushed between steps.  The same
+line carries the roofline of the attend kernel, an end-to-end figure through host
+buffers, a sweep of independent queries per sequence, causal prefill tokens/s
+(524K + 8K chunk, and 1M + 8K), the 2M-token tree build in GB/s, 2M decode latency
+and the fp64 oracle timed on the host cores.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--quick]
+
+With --gpus N > 1 it runs under torchrun, one rank per GPU: every rank decodes its
+own 4 sequences (weak scaling, no data-path collective); the timed region is
+bracketed by barriers and the maximum over ranks is reported.
+"""
+
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import recsa_inputs as I  # noqa: E402
+
+METRIC = "RecSA decode queries/s & prefill tokens/s at 1M ctx; achieved HBM GB/s vs peak"
+ROW = 256  # bytes of one bf16 row of 128
+FLUSH_BYTES = 256 << 20  # > 126 MB L2
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), float(d.get("bf16_tflops", 0)), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed work runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.idx = device_index
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(device_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        busy = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": max(mx) if mx else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------- timing
+
+class Timer:
+    """Per-step CUDA-event timing on the launching stream, L2 flushed before each step."""
+
+    def __init__(self, dist_on: bool):
+        self.dist_on = dist_on
+        self.flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    def flush(self):
+        self.flush_buf.zero_()
+
+    def barrier(self):
+        if self.dist_on:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def run(self, fn, steps: int, warmup: int, flush: bool = True):
+        for _ in range(warmup):
+            if flush:
+                self.flush()
+            fn()
+        stream = torch.cuda.current_stream()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        self.barrier()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for a, b in ev:
+            if flush:
+                self.flush()
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        self.barrier()
+        wall = time.perf_counter() - t0
+        per = [a.elapsed_time(b) / 1e3 for a, b in ev]
+        return per, wall
+
+
+def max_over_ranks(x: float, dist_on: bool) -> float:
+    if not dist_on:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def pct(xs, q):
+    s = sorted(xs)
+    return s[min(len(s) - 1, max(0, int(round(q * (len(s) - 1)))))]
+
+
+# ----------------------------------------------------------------------------- legs
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "hierarchical_sparse_attention_build_b200", "csrc")
+    for f in ("recsa_attend.cu", "recsa_device.cuh", "recsa_internal.h"):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(name: str):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the current kernel source."""
+    path = os.path.join(ROOT, "profiles", f"{name}.txt")
+    try:
+        kv = dict(line.split(":", 1) for line in open(path) if ":" in line)
+        if kv.get("kernel_source_sha256", "").strip() != kernel_source_sha():
+            return None
+        return float(kv["dram_bytes_per_launch"].strip())
+    except Exception:
+        return None
+
+
+def make_tree(R, p, inp, length, build=True):
+    tree = R.RecsaTree(p, inp["k_tok"], inp["v_tok"], inp["pooler"], length)
+    ws = R.Workspace(p, tree.capacity, "cuda")
+    if build:
+        R.build_tree(p, tree)
+    return tree, ws
+
+
+def decode_entries(R, p, tree, ws, q):
+    B, Q, Hq, _ = q.shape
+    tiles = B * p.num_kv_heads * Q
+    ent = torch.zeros(tiles, 2, dtype=torch.int32, device="cuda")
+    out = torch.empty(B, Q, Hq, 128, dtype=torch.bfloat16, device="cuda")
+    R.decode(p, tree, q, out, ws, entries=ent)
+    R.check_device_errors(ws)
+    return int(ent.sum().item())
+
+
+def leg_decode_1m(R, timer, args, dist_on, hbm_peak, peaks_src):
+    w = I.WORKLOADS["decode_1m"]
+    inp = I.decode_inputs(w, device="cuda")
+    p = R.params(num_kv_heads=w.kv_heads, num_q_heads=w.q_heads, branching=w.branching, top_k=w.top_k)
+    tree, ws = make_tree(R, p, inp, w.length)
+    q = inp["q"]
+    B, Q, Hq, _ = q.shape
+    out = torch.empty(B, Q, Hq, 128, dtype=torch.bfloat16, device="cuda")
+    rows = decode_entries(R, p, tree, ws, q)
+    bytes_per_launch = rows * ROW + q.numel() * 2 + out.numel() * 2
+    torch.cuda.synchronize()
+
+    per, wall = timer.run(lambda: R.decode(p, tree, q, out, ws), args.steps, args.warmup)
+    total = max_over_ranks(sum(per), dist_on)
+    mean_s = total / args.steps
+    res = dict(per_step_s=per, total_s=total, wall_s=wall, mean_s=mean_s, rows=rows,
+               bytes_per_launch=bytes_per_launch, queries=B * Q)
+
+    # end to end: pinned host query in, pinned host output back, every step
+    q_host = q.cpu().pin_memory()
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    q_dev = torch.empty_like(q)
+
+    def e2e_step():
+        q_dev.copy_(q_host, non_blocking=True)
+        R.decode(p, tree, q_dev, out, ws)
+        out_host.copy_(out, non_blocking=True)
+
+    per_e, _ = timer.run(e2e_step, args.steps, args.warmup)
+    res["e2e_total_s"] = max_over_ranks(sum(per_e), dist_on)
+    res["h2d"] = q_host.numel() * 2
+    res["d2h"] = out_host.numel() * 2
+
+    # independent decode queries per sequence (throughput regime), same caches
+    sweep = []
+    for nq in ([1, 4, 16, 64] if not args.quick else [1, 16]):
+        g = torch.Generator(device="cuda").manual_seed(77 + nq)
+        qs = torch.randn(B, nq, Hq, 128, generator=g, device="cuda").to(torch.bfloat16)
+        outs = torch.empty(B, nq, Hq, 128, dtype=torch.bfloat16, device="cuda")
+        r = decode_entries(R, p, tree, ws, qs)
+        nb = r * ROW + qs.numel() * 2 + outs.numel() * 2
+        st = max(20, args.steps // (4 * nq))
+        per_s, _ = timer.run(lambda: R.decode(p, tree, qs, outs, ws), st, max(3, args.warmup // 4))
+        t = max_over_ranks(sum(per_s), dist_on) / st
+        sweep.append({"queries_per_seq": nq, "queries_per_s": B * nq / t, "us_per_call": t * 1e6,
+                      "logical_GBps": nb / t / 1e9, "frac": nb / t / 1e9 / hbm_peak})
+    res["sweep"] = sweep
+    R.check_device_errors(ws)
+    del tree, ws, inp, q, out
+    torch.cuda.empty_cache()
+    return res, w
+
+
+def leg_prefill(R, timer, args, dist_on, hbm_peak, name, length):
+    base = I.WORKLOADS["prefill_524k"]
+    w = dataclasses.replace(base, name=name, length=length)
+    inp = I.prefill_inputs(w, device="cuda")
+    p = R.params(num_kv_heads=w.kv_heads, num_q_heads=w.q_heads, branching=w.branching, top_k=w.top_k)
+    tree, ws = make_tree(R, p, inp, w.length)
+    k_new, v_new, q = inp["k_new"], inp["v_new"], inp["q"]
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
+    tiles = w.batch * w.kv_heads * w.chunk
+    ent = torch.zeros(tiles, 2, dtype=torch.int32, device="cuda")
+
+    def step(entries=None):
+        tree.length = w.length  # the call appends at L; every step redoes the same chunk
+        R.prefill_chunk(p, tree, k_new, v_new, q, out, ws, entries=entries)
+
+    step(ent)
+    R.check_device_errors(ws)
+    rows = int(ent.sum().item())
+    append_bytes = 2 * 2 * k_new.numel() * 2  # read chunk K/V, write into the caches
+    nodes_touched = 0
+    span = w.branching
+    for _ in range(tree.levels):
+        nodes_touched += -(-(w.length + w.chunk) // span) - w.length // span
+        span *= w.branching
+    ext_bytes = nodes_touched * w.kv_heads * w.batch * ROW * 2 * (w.branching + 1)
+    logical = rows * ROW + q.numel() * 2 + out.numel() * 2 + append_bytes + ext_bytes
+    steps = max(5, args.steps // 200) if not args.quick else 5
+    per, _ = timer.run(step, steps, 2)
+    t = max_over_ranks(sum(per), dist_on) / steps
+    R.check_device_errors(ws)
+    del tree, ws, inp
+    torch.cuda.empty_cache()
+    return {"workload": f"{name}: B={w.batch}, L={w.length} cached + C={w.chunk} chunk, Hq={w.q_heads}, "
+                        f"Hkv={w.kv_heads}, b={w.branching}, k={w.top_k}",
+            "tokens_per_s": w.batch * w.chunk / t, "ms_per_chunk": t * 1e3,
+            "rows_read": rows, "logical_bytes": logical, "logical_GBps": logical / t / 1e9,
+            "logical_frac_of_hbm": logical / t / 1e9 / hbm_peak,
+            "note": "append + extension build + causal attend per call; rows re-read by neighbouring "
+                    "queries hit L2, so logical GB/s can exceed HBM bandwidth"}
+
+
+def leg_build_2m(R, timer, args, dist_on, hbm_peak):
+    w = I.WORKLOADS["build_decode_2m"]
+    inp = I.decode_inputs(w, device="cuda")
+    p = R.params(num_kv_heads=w.kv_heads, num_q_heads=w.q_heads, branching=w.branching, top_k=w.top_k)
+    tree, ws = make_tree(R, p, inp, w.length, build=False)
+    tok_bytes = 2 * inp["k_tok"].numel() * 2
+    node_rows = 0
+    n = w.length
+    while n > w.branching:
+        n = -(-n // w.branching)
+        node_rows += n
+    node_bytes = 2 * node_rows * w.kv_heads * w.batch * ROW
+    algorithmic = tok_bytes + node_bytes  # every token read once, every node written once
+    steps = max(5, args.steps // 500) if not args.quick else 3
+    per, _ = timer.run(lambda: R.build_tree(p, tree), steps, 2)
+    t = max_over_ranks(sum(per), dist_on) / steps
+    q = inp["q"]
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
+    rows = decode_entries(R, p, tree, ws, q)
+    per_d, _ = timer.run(lambda: R.decode(p, tree, q, out, ws), max(50, args.steps // 4), args.warmup)
+    R.check_device_errors(ws)
+    del tree, ws, inp
+    torch.cuda.empty_cache()
+    return {"workload": f"build_decode_2m: B=1, L={w.length}, Hkv=8, b=16 (build); decode B=1, k=8",
+            "build_ms": t * 1e3, "build_GBps": algorithmic / t / 1e9, "build_frac": algorithmic / t / 1e9 / hbm_peak,
+            "build_bytes": algorithmic,
+            "decode_latency_us": {"median": statistics.median(per_d) * 1e6, "p10": pct(per_d, 0.1) * 1e6,
+                                  "p90": pct(per_d, 0.9) * 1e6},
+            "decode_rows": rows}
+
+
+# ----------------------------------------------------------------------------- oracle (CPU baseline)
+
+def oracle_decode_rate(budget_s: float, device_inputs=None, max_tiles=None, warmup_tiles=0):
+    """The fp64 oracle's decode rate on a bounded sample of the 1M workload.
+
+    Sample: one sequence, two KV groups of the decode_1m recipe; their trees are built
+    first (untimed, like the GPU leg, which decodes over a tree built beforehand), then
+    the oracle attends as many query groups as fit in `budget_s`.  A decode query of the
+    workload is 8 such tiles (one per KV group), so queries/s = tiles/s / 8."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import recsa_oracle as O
+
+    w = I.WORKLOADS["decode_1m"]
+    if device_inputs is not None:
+        kb = I.bf16_bits(device_inputs["k_tok"][0, :2])
+        vb = I.bf16_bits(device_inputs["v_tok"][0, :2])
+        qb = I.bf16_bits(device_inputs["q"][0:1])
+        W = device_inputs["pooler"].double().cpu().numpy()
+        src = "slices of the GPU leg's seeded cache (sequence 0, KV heads 0-1)"
+    else:
+        small = dataclasses.replace(w, batch=1, kv_heads=2, q_heads=8)
+        inp = I.decode_inputs(small, device="cpu")
+        kb, vb, qb = I.bf16_bits(inp["k_tok"][0]), I.bf16_bits(inp["v_tok"][0]), I.bf16_bits(inp["q"])
+        W = inp["pooler"].double().numpy()
+        src = "the decode_1m recipe drawn on the CPU for 1 sequence x 2 KV heads"
+    with threadpool_limits(limits=1):
+        t_build = time.perf_counter()
+        trees = [O.build_tree(O.bf16_bits_to_f64(kb[h, :w.length]), O.bf16_bits_to_f64(vb[h, :w.length]), W,
+                              w.branching) for h in range(2)]
+        t_build = time.perf_counter() - t_build
+        g = torch.Generator().manual_seed(5)
+        for i in range(warmup_tiles):  # untimed
+            O.attend(torch.randn(4, 128, generator=g, dtype=torch.float64).numpy(), trees[i % 2], w.length, w.top_k)
+        tiles = 0
+        t0 = time.perf_counter()
+        while True:
+            h = tiles % 2
+            if tiles < 2:
+                q = O.bf16_bits_to_f64(qb[0, 0, h * 4:(h + 1) * 4])
+            else:
+                q = torch.randn(4, 128, generator=g, dtype=torch.float64).numpy()
+            O.attend(q, trees[h], w.length, w.top_k)
+            tiles += 1
+            el = time.perf_counter() - t0
+            if el >= budget_s or (max_tiles and tiles >= max_tiles):
+                break
+    return {"tiles": tiles, "seconds": el, "queries_per_s": tiles / 8 / el, "tree_build_s": t_build,
+            "source": src}
+
+
+# ----------------------------------------------------------------------------- arms
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    # every step is one tile of the oracle on the host; K + W steps bounded to a few minutes
+    steps, warmup = args.steps, args.warmup
+    budget = None
+    r = oracle_decode_rate(budget_s=1e9, max_tiles=steps, warmup_tiles=warmup) if steps + warmup <= 20000 else None
+    if r is None:
+        budget = 120.0
+        r = oracle_decode_rate(budget_s=budget)
+    value = r["queries_per_s"]
+    w = I.WORKLOADS["decode_1m"]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": args.gpus,
+        "steps": steps, "warmup": warmup, "ms_per_step": r["seconds"] / max(r["tiles"], 1) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"decode_1m: B={w.batch}, L={w.length}, Hq={w.q_heads}, Hkv={w.kv_heads}, d=128, "
+                               f"b={w.branching}, k={w.top_k}, Q=1", "batch": w.batch, "seq_len": w.length,
+                   "parallelism": "none (host oracle)"},
+        "cpu_baseline": {"value": value, "unit": "queries/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{r['tiles']} query-group tiles (1 step = 1 tile) over trees of 2 KV heads of "
+                                   f"{r['source']}; trees built untimed in {r['tree_build_s']:.1f} s; "
+                                   "queries/s = tiles/s / 8"},
+        "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_profile_case(args):
+    """Small case of one kernel for an ncu capture (a few launches, about 1 GB on the device).
+
+    decode: the 1M-context decode tile structure of the headline (b = 16, k = 8, needles)
+    with 1 sequence and 2 KV groups (2 tiles per launch instead of 32)."""
+    import hierarchical_sparse_attention_build_b200 as R
+
+    torch.cuda.set_device(0)
+    if args.profile == "decode":
+        w = dataclasses.replace(I.WORKLOADS["decode_1m"], batch=1, kv_heads=2, q_heads=8)
+        inp = I.decode_inputs(w, device="cuda")
+        p = R.params(num_kv_heads=w.kv_heads, num_q_heads=w.q_heads, branching=w.branching, top_k=w.top_k)
+        tree, ws = make_tree(R, p, inp, w.length)
+        out = torch.empty(inp["q"].shape, dtype=torch.bfloat16, device="cuda")
+        flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        for _ in range(6):
+            flush.zero_()
+            R.decode(p, tree, inp["q"], out, ws)
+        R.check_device_errors(ws)
+        rows = decode_entries(R, p, tree, ws, inp["q"])
+        print(json.dumps({"profile": "decode", "tiles": w.batch * w.kv_heads, "rows_per_launch": rows,
+                          "kernel_source_sha256": kernel_source_sha()}))
+    elif args.profile == "prefill":
+        w = dataclasses.replace(I.WORKLOADS["prefill_524k"], length=65536, chunk=1024)
+        inp = I.prefill_inputs(w, device="cuda")
+        p = R.params(num_kv_heads=w.kv_heads, num_q_heads=w.q_heads, branching=w.branching, top_k=w.top_k)
+        tree, ws = make_tree(R, p, inp, w.length)
+        out = torch.empty(inp["q"].shape, dtype=torch.bfloat16, device="cuda")
+        for _ in range(4):
+            tree.length = w.length
+            R.prefill_chunk(p, tree, inp["k_new"], inp["v_new"], inp["q"], out, ws)
+        R.check_device_errors(ws)
+        print(json.dumps({"profile": "prefill", "length": w.length, "chunk": w.chunk,
+                          "tiles": w.batch * w.kv_heads * w.chunk, "kernel_source_sha256": kernel_source_sha()}))
+    elif args.profile == "build":
+        w = dataclasses.replace(I.WORKLOADS["build_decode_2m"], length=1 << 19)
+        inp = I.decode_inputs(w, device="cuda")
+        p = R.params(num_kv_heads=w.kv_heads, num_q_heads=w.q_heads, branching=w.branching, top_k=w.top_k)
+        tree, ws = make_tree(R, p, inp, w.length, build=False)
+        for _ in range(4):
+            R.build_tree(p, tree)
+        torch.cuda.synchronize()
+        print(json.dumps({"profile": "build", "length": w.length, "kv_heads": w.kv_heads}))
+    torch.cuda.synchronize()
+
+
+def run_gpu(args):
+    import hierarchical_sparse_attention_build_b200 as R
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist_on = world > 1
+    torch.cuda.set_device(local)
+    if dist_on:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    hbm_peak, _, peaks_src = load_peaks()
+    timer = Timer(dist_on)
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES")
+    clocks = ClockSampler(visible.split(",")[local].strip() if visible else local)
+    dec, w = leg_decode_1m(R, timer, args, dist_on, hbm_peak, peaks_src)
+    extra = {}
+    if not args.headline_only:
+        extra["prefill"] = leg_prefill(R, timer, args, dist_on, hbm_peak, "prefill_524k", 524288)
+        extra["prefill_1m"] = leg_prefill(R, timer, args, dist_on, hbm_peak, "prefill_1m", 1 << 20)
+        extra["build_2m"] = leg_build_2m(R, timer, args, dist_on, hbm_peak)
+    clk = clocks.stop()
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        r = oracle_decode_rate(budget_s=args.cpu_seconds)
+        cpu = {"value": r["queries_per_s"], "unit": "queries/s", "cores": 1, "kind": "oracle",
+               "sample": f"{r['tiles']} query-group tiles in {r['seconds']:.1f} s over the trees of 2 KV heads of "
+                         f"{r['source']} (trees built untimed, {r['tree_build_s']:.1f} s); queries/s = tiles/s / 8; "
+                         "numpy limited to 1 thread"}
+    if dist_on:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    B = w.batch
+    n = world
+    value = n * dec["queries"] * args.steps / dec["total_s"]
+    mean_s = dec["mean_s"]
+    achieved = dec["bytes_per_launch"] / mean_s / 1e9
+    traffic = recorded_traffic("decode_1m_attend_traffic")
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "queries/s",
+        "n_gpus": n,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": mean_s * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": f"decode_1m: B={B}, L={w.length}, Hq={w.q_heads}, Hkv={w.kv_heads}, d=128, "
+                               f"b={w.branching}, k={w.top_k}, Q=1 query per sequence, needles=64 (bf16 K/V, "
+                               "fp32 accumulation, bf16 output)",
+                   "global_batch": B * n, "seq_len": w.length, "parallelism": f"replicas x{n} (no collective)",
+                   "l2": "flushed between timed steps (256 MiB write, untimed)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": traffic,
+                     "kernel": "attend_kernel<4,4> (recsa_decode)",
+                     "algorithmic_bytes_per_launch": dec["bytes_per_launch"],
+                     "peak_source": f"{peaks_src} hbm_gbs (MEASURED_PEAKS.json)"},
+        "e2e": {"value": n * dec["queries"] * args.steps / dec["e2e_total_s"], "unit": "queries/s",
+                "h2d_bytes_per_step": dec["h2d"], "d2h_bytes_per_step": dec["d2h"]},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+        "decode": {"us_per_step_median": statistics.median(dec["per_step_s"]) * 1e6,
+                   "us_per_step_p10": pct(dec["per_step_s"], 0.1) * 1e6,
+                   "us_per_step_p90": pct(dec["per_step_s"], 0.9) * 1e6,
+                   "rows_read_per_call": dec["rows"], "queries_per_seq_sweep": dec["sweep"]},
+        "cpu_baseline": cpu,
+    }
+    line.update(extra)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--quick", action="store_true", help="fewer sweep points and steps in the side legs")
+    ap.add_argument("--headline-only", action="store_true", help="skip the prefill and build legs")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--profile", choices=["decode", "prefill", "build"], help="run a small case of one kernel for ncu")
+    args = ap.parse_args()
+    if args.profile:
+        run_profile_case(args)
+        return
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

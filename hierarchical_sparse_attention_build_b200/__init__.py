@@ -68,10 +68,15 @@ class Tree(ctypes.Structure):
 class Debug(ctypes.Structure):
     _fields_ = [
         ("sel_idx", ctypes.c_void_p),
-        ("sel_levels", ctypes.c_int32),
-        ("cluster_size", ctypes.c_int32),
         ("entries", ctypes.c_void_p),
+        ("sel_levels", ctypes.c_int32),
+        ("kernel", ctypes.c_int32),
+        ("cluster_size", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
     ]
+
+
+KERNEL_AUTO, KERNEL_CTA, KERNEL_WARP = 0, 1, 2
 
 
 def _load() -> ctypes.CDLL:
@@ -203,19 +208,19 @@ def build_tree(p: Params, tree: RecsaTree, stream=None) -> None:
     _check(_lib.recsa_build_tree(ctypes.byref(p), ctypes.byref(tree.c), _stream(stream)))
 
 
-def _debug(sel_idx=None, sel_levels=0, cluster_size=0, entries=None):
-    if sel_idx is None and entries is None and cluster_size == 0:
+def _debug(sel_idx=None, sel_levels=0, cluster_size=0, entries=None, kernel=0):
+    if sel_idx is None and entries is None and cluster_size == 0 and kernel == 0:
         return None
-    return Debug(sel_idx.data_ptr() if sel_idx is not None else None, sel_levels, cluster_size,
-                 entries.data_ptr() if entries is not None else None)
+    return Debug(sel_idx.data_ptr() if sel_idx is not None else None,
+                 entries.data_ptr() if entries is not None else None, sel_levels, kernel, cluster_size, 0)
 
 
 def decode(p: Params, tree: RecsaTree, q: torch.Tensor, out: torch.Tensor, ws: Workspace, sel_idx=None,
-           sel_levels: int = 0, entries=None, cluster_size: int = 0, stream=None) -> None:
+           sel_levels: int = 0, entries=None, cluster_size: int = 0, kernel: int = 0, stream=None) -> None:
     """recsa_decode: q [B][Q][Hq][128] bf16 -> out [B][Q][Hq][128] (fp32 or bf16)."""
     assert q.dtype == torch.bfloat16 and q.is_contiguous() and out.is_contiguous()
     nq = q.shape[1]
-    dbg = _debug(sel_idx, sel_levels, cluster_size, entries)
+    dbg = _debug(sel_idx, sel_levels, cluster_size, entries, kernel)
     _check(_lib.recsa_decode(ctypes.byref(p), ctypes.byref(tree.c), _ptr(q), nq, _ptr(out),
                              int(out.dtype == torch.float32), _ptr(ws.buf), ws.nbytes,
                              ctypes.byref(dbg) if dbg is not None else None, _stream(stream)))
@@ -223,12 +228,12 @@ def decode(p: Params, tree: RecsaTree, q: torch.Tensor, out: torch.Tensor, ws: W
 
 def prefill_chunk(p: Params, tree: RecsaTree, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor,
                   out: torch.Tensor, ws: Workspace, sel_idx=None, sel_levels: int = 0, entries=None,
-                  cluster_size: int = 0, stream=None) -> None:
+                  cluster_size: int = 0, kernel: int = 0, stream=None) -> None:
     """recsa_prefill_chunk: append [B][C][Hkv][128] K/V, extend the tree, attend the C queries causally."""
     for t in (k_new, v_new, q):
         assert t.dtype == torch.bfloat16 and t.is_contiguous()
     chunk = q.shape[1]
-    dbg = _debug(sel_idx, sel_levels, cluster_size, entries)
+    dbg = _debug(sel_idx, sel_levels, cluster_size, entries, kernel)
     _check(_lib.recsa_prefill_chunk(ctypes.byref(p), ctypes.byref(tree.c), _ptr(k_new), _ptr(v_new), _ptr(q), chunk,
                                     _ptr(out), int(out.dtype == torch.float32), _ptr(ws.buf), ws.nbytes,
                                     ctypes.byref(dbg) if dbg is not None else None, _stream(stream)))

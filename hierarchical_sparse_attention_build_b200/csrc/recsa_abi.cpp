@@ -158,6 +158,7 @@ recsa_status check_debug(const recsa_params *p, const recsa_debug *d) {
     return fail(RECSA_ERR_INVALID_ARGUMENT, "sel_idx needs 1 <= top_k <= %d and sel_levels >= 1", kDebugMaxK);
   if (d->cluster_size != 0 && d->cluster_size != 1 && d->cluster_size != 2 && d->cluster_size != 4)
     return fail(RECSA_ERR_INVALID_ARGUMENT, "cluster_size %d (0, 1, 2 or 4)", d->cluster_size);
+  if (d->kernel < 0 || d->kernel > 2) return fail(RECSA_ERR_INVALID_ARGUMENT, "kernel %d (0, 1 or 2)", d->kernel);
   return RECSA_OK;
 }
 
@@ -279,6 +280,7 @@ RECSA_API recsa_status recsa_decode(const recsa_params *params, const recsa_tree
   l.table_rows_needed = (int)mc + 1;
   l.max_cand = (int)((mc + 31) / 32 * 32);
   l.cluster_size = debug ? debug->cluster_size : 0;
+  l.kernel = debug ? debug->kernel : 0;
   l.debug = debug;
   const int rc = launch_attend(l, stream);
   if (rc != 0) return cuda_fail(rc, "decode attend");
@@ -333,6 +335,7 @@ RECSA_API recsa_status recsa_prefill_chunk(const recsa_params *params, recsa_tre
   l.table_rows_needed = (int)mc + 1;
   l.max_cand = (int)((mc + 31) / 32 * 32);
   l.cluster_size = debug ? debug->cluster_size : 0;
+  l.kernel = debug ? debug->kernel : 0;
   l.debug = debug;
   rc = launch_attend(l, stream);
   if (rc != 0) return cuda_fail(rc, "prefill attend");

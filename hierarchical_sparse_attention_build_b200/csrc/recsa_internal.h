@@ -72,6 +72,7 @@ struct AttendLaunch {
   int table_rows_needed;
   int max_cand;        // candidate buffer size per level (multiple of 32)
   int cluster_size;    // 0 = automatic
+  int kernel;          // 0 = automatic, 1 = CTA/cluster per tile, 2 = warp per tile
   const recsa_debug *debug;
 };
 int launch_attend(const AttendLaunch &a, void *stream);

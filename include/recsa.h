@@ -110,19 +110,23 @@ typedef struct recsa_tree {
   const float *pooler;
 } recsa_tree;
 
-/* Optional diagnostics of recsa_decode / recsa_prefill_chunk (pass NULL for none).
- * A "tile" is one (sequence, query, KV group); tiles are numbered
- * ((s * Hkv + g) * num_queries + query).
+/* Optional diagnostics and launch-shape overrides of recsa_decode / recsa_prefill_chunk
+ * (pass NULL for none).  A "tile" is one (sequence, query, KV group); tiles are
+ * numbered ((s * Hkv + g) * num_queries + query).
  *   sel_idx  : int32 [tiles][sel_levels][top_k]; slot (l-1) receives the node indices
  *              kept at level l (ascending, -1 padded).  Needs top_k <= 64.
  *   entries  : int32 [tiles][2]; keys scored and values folded by the tile (rows read).
- *   cluster_size: 0 = automatic; 1, 2 or 4 forces the number of CTAs that share one
- *              tile (a launch-shape choice; results are identical up to rounding). */
+ *   kernel   : 0 = automatic; 1 = one CTA (or a cluster of cluster_size CTAs) per tile,
+ *              the low-latency shape for few tiles; 2 = one warp per tile, the
+ *              throughput shape for many tiles.  Results agree up to fp32 rounding.
+ *   cluster_size: with kernel 1: 0 = automatic, or 1, 2, 4 CTAs per tile. */
 typedef struct recsa_debug {
   int32_t *sel_idx;
-  int32_t sel_levels;
-  int32_t cluster_size;
   int32_t *entries;
+  int32_t sel_levels;
+  int32_t kernel;
+  int32_t cluster_size;
+  int32_t reserved;
 } recsa_debug;
 
 /* Arena layout of a tree of `capacity` token slots (host only, no CUDA call).

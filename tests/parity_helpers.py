@@ -77,7 +77,7 @@ class GpuCase:
     def build(self):
         R.build_tree(self.p, self.tree)
 
-    def decode(self, q: torch.Tensor, cluster_size=0, sel_levels=None, fp32=True):
+    def decode(self, q: torch.Tensor, cluster_size=0, sel_levels=None, fp32=True, kernel=0):
         q = q.to(self.k_tok.device).contiguous()
         B, Q, Hq, _ = q.shape
         out = torch.empty(B, Q, Hq, 128, dtype=torch.float32 if fp32 else torch.bfloat16, device=q.device)
@@ -88,12 +88,12 @@ class GpuCase:
             sel = torch.full((tiles, lv, self.p.top_k), -7, dtype=torch.int32, device=q.device)
         ent = torch.zeros(tiles, 2, dtype=torch.int32, device=q.device)
         R.decode(self.p, self.tree, q, out, self.ws, sel_idx=sel, sel_levels=lv, entries=ent,
-                 cluster_size=cluster_size)
+                 cluster_size=cluster_size, kernel=kernel)
         R.check_device_errors(self.ws)
         torch.cuda.synchronize()
         return out.cpu(), (sel.cpu().numpy() if sel is not None else None), ent.cpu().numpy()
 
-    def prefill(self, k_new, v_new, q, cluster_size=0, fp32=True, sel_levels=None):
+    def prefill(self, k_new, v_new, q, cluster_size=0, fp32=True, sel_levels=None, kernel=0):
         dev = self.k_tok.device
         k_new, v_new, q = k_new.to(dev).contiguous(), v_new.to(dev).contiguous(), q.to(dev).contiguous()
         B, C, Hq, _ = q.shape
@@ -105,7 +105,7 @@ class GpuCase:
             sel = torch.full((tiles, lv, self.p.top_k), -7, dtype=torch.int32, device=dev)
         ent = torch.zeros(tiles, 2, dtype=torch.int32, device=dev)
         R.prefill_chunk(self.p, self.tree, k_new, v_new, q, out, self.ws, sel_idx=sel, sel_levels=lv, entries=ent,
-                        cluster_size=cluster_size)
+                        cluster_size=cluster_size, kernel=kernel)
         R.check_device_errors(self.ws)
         torch.cuda.synchronize()
         return out.cpu(), (sel.cpu().numpy() if sel is not None else None), ent.cpu().numpy()

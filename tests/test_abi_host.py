@@ -118,11 +118,12 @@ def test_decode_bad_call_arguments_rejected():
     assert _decode(p, t, nq=0) == INVALID
     assert _decode(p, t, ws=0) == INVALID
     assert _decode(p, t, ws_bytes=100) == WS_SMALL
-    assert _decode(_p(top_k=65), t, dbg=R.Debug(FAKE, 4, 0, 0), ws_bytes=100) == WS_SMALL
+    assert _decode(_p(top_k=65), t, dbg=R.Debug(FAKE, 0, 4, 0, 0, 0), ws_bytes=100) == WS_SMALL
     p65 = _p(top_k=65)
     ws = R.workspace_size(p65, 4096)
-    assert _decode(p65, t, dbg=R.Debug(FAKE, 4, 0, 0), ws_bytes=ws) == INVALID
-    assert _decode(p, t, dbg=R.Debug(0, 0, 3, 0), ws_bytes=R.workspace_size(p, 4096)) == INVALID
+    assert _decode(p65, t, dbg=R.Debug(FAKE, 0, 4, 0, 0, 0), ws_bytes=ws) == INVALID
+    assert _decode(p, t, dbg=R.Debug(0, 0, 0, 0, 3, 0), ws_bytes=R.workspace_size(p, 4096)) == INVALID
+    assert _decode(p, t, dbg=R.Debug(0, 0, 0, 5, 0, 0), ws_bytes=R.workspace_size(p, 4096)) == INVALID
     # k = all at a long context needs more candidates per level than the kernel holds
     pall = _p(top_k=R.TOPK_ALL)
     big = _tree(capacity=1 << 16, length=1 << 16)

@@ -38,8 +38,12 @@ def _compare_build(case: GpuCase, trees, b):
     return mism, total
 
 
-def _decode_and_check(case, trees, q, k, cluster_size=0, isolated=False):
-    out, sel, ent = case.decode(q, cluster_size=cluster_size)
+# launch shapes: (kernel, cluster_size); kernel 1 = CTA/cluster per tile, 2 = warp per tile
+SHAPES = [(1, 1), (1, 2), (1, 4), (2, 0)]
+
+
+def _decode_and_check(case, trees, q, k, cluster_size=0, kernel=0):
+    out, sel, ent = case.decode(q, cluster_size=cluster_size, kernel=kernel)
     p = case.p
     G = p.num_q_heads // p.num_kv_heads
     B, Q = q.shape[:2]
@@ -80,14 +84,15 @@ def test_build_odd_shapes_match_oracle_rows(B, hkv, L, cap, b):
     print(f"build: {mism} of {total} elements not bit-identical")
 
 
-@pytest.mark.parametrize("cluster_size", [0, 1, 2, 4])
-def test_decode_tiny_end_to_end(cluster_size):
+@pytest.mark.parametrize("kernel,cluster_size", [(0, 0)] + SHAPES)
+def test_decode_tiny_end_to_end(kernel, cluster_size):
     w = I.WORKLOADS["tiny_decode"]
     inp = I.decode_inputs(w)
     case = GpuCase(inp, _params(1, 4, w.branching, w.top_k), w.length)
     case.build()
-    stats = _decode_and_check(case, oracle_trees(inp, w.branching, w.length), inp["q"], w.top_k, cluster_size)
-    print("tiny decode", stats)
+    stats = _decode_and_check(case, oracle_trees(inp, w.branching, w.length), inp["q"], w.top_k, cluster_size,
+                              kernel)
+    print("tiny decode", kernel, cluster_size, stats)
 
 
 def test_decode_tiny_attend_on_oracle_tree():
@@ -106,12 +111,13 @@ def test_decode_tiny_attend_on_oracle_tree():
     print("tiny attend on oracle tree", stats)
 
 
-def test_decode_topk_all_equals_dense_attention():
+@pytest.mark.parametrize("kernel,cluster_size", SHAPES)
+def test_decode_topk_all_equals_dense_attention(kernel, cluster_size):
     w = I.WORKLOADS["tiny_decode"]
     inp = I.decode_inputs(w)
     case = GpuCase(inp, _params(1, 4, w.branching, R.TOPK_ALL), w.length)
     case.build()
-    out, _, ent = case.decode(inp["q"])
+    out, _, ent = case.decode(inp["q"], cluster_size=cluster_size, kernel=kernel)
     kt, vt = O.bf16_bits_to_f64(bits(inp["k_tok"])[0, 0]), O.bf16_bits_to_f64(bits(inp["v_tok"])[0, 0])
     qb = bits(inp["q"])
     stats = Stats()
@@ -123,12 +129,13 @@ def test_decode_topk_all_equals_dense_attention():
     print("k=all vs dense", stats)
 
 
-def test_decode_k0_is_attention_over_top_summaries():
+@pytest.mark.parametrize("kernel,cluster_size", SHAPES)
+def test_decode_k0_is_attention_over_top_summaries(kernel, cluster_size):
     w = I.WORKLOADS["tiny_decode"]
     inp = I.decode_inputs(w)
     case = GpuCase(inp, _params(1, 4, w.branching, 0), w.length)
     case.build()
-    out, _, _ = case.decode(inp["q"])
+    out, _, _ = case.decode(inp["q"], cluster_size=cluster_size, kernel=kernel)
     t = oracle_trees(inp, w.branching, w.length)[0][0]
     qb = bits(inp["q"])
     stats = Stats()
@@ -148,43 +155,45 @@ def test_decode_k0_is_attention_over_top_summaries():
     (1, 2, 4, 3000, 5, 40, 1),     # many candidates per level (several gather chunks)
     (2, 1, 4, 2048, 4, 1, 4),      # k = 1
 ])
-@pytest.mark.parametrize("cluster_size", [1, 4])
-def test_decode_odd_shapes(B, hkv, G, L, b, k, Q, cluster_size):
+@pytest.mark.parametrize("kernel,cluster_size", [(1, 1), (1, 4), (2, 0)])
+def test_decode_odd_shapes(B, hkv, G, L, b, k, Q, kernel, cluster_size):
     inp = I.random_case(B, L, hkv, hkv * G, Q, seed=7 * L + b)
     case = GpuCase(inp, _params(hkv, G, b, k), L)
     case.build()
-    _decode_and_check(case, oracle_trees(inp, b, L), inp["q"], k, cluster_size)
+    _decode_and_check(case, oracle_trees(inp, b, L), inp["q"], k, cluster_size, kernel)
 
 
-def test_decode_ties_keep_lower_index():
+@pytest.mark.parametrize("kernel,cluster_size", SHAPES)
+def test_decode_ties_keep_lower_index(kernel, cluster_size):
     L, b, k = 4096, 8, 3
     inp = I.random_case(1, L, 1, 4, 2, seed=3)
     inp["k_tok"].zero_()  # every score is exactly 0
     case = GpuCase(inp, _params(1, 4, b, k), L)
     case.build()
-    _, sel, _ = case.decode(inp["q"])
+    _, sel, _ = case.decode(inp["q"], cluster_size=cluster_size, kernel=kernel)
     for tile in range(2):
         for lvl_sel in gpu_selection(sel, tile, 3):
             assert lvl_sel == [0, 1, 2]
 
 
-def test_decode_bf16_output_is_rounded_fp32_output():
+@pytest.mark.parametrize("kernel", [1, 2])
+def test_decode_bf16_output_is_rounded_fp32_output(kernel):
     w = I.WORKLOADS["tiny_decode"]
     inp = I.decode_inputs(w)
     case = GpuCase(inp, _params(1, 4, w.branching, w.top_k), w.length)
     case.build()
-    o32, _, _ = case.decode(inp["q"])
-    o16, _, _ = case.decode(inp["q"], fp32=False)
+    o32, _, _ = case.decode(inp["q"], kernel=kernel)
+    o16, _, _ = case.decode(inp["q"], fp32=False, kernel=kernel)
     assert torch.equal(o32.to(torch.bfloat16), o16)
 
 
-def _prefill_check(B, hkv, G, L, C, b, k, cluster_size=0, seed=1):
+def _prefill_check(B, hkv, G, L, C, b, k, cluster_size=0, seed=1, kernel=0):
     cap = L + C
     inp = I.random_case(B, L, hkv, hkv * G, 0, seed=seed, capacity=cap, chunk=C)
     case = GpuCase(inp, _params(hkv, G, b, k), L)
     if L:
         case.build()
-    out, sel, ent = case.prefill(inp["k_new"], inp["v_new"], inp["q"], cluster_size=cluster_size)
+    out, sel, ent = case.prefill(inp["k_new"], inp["v_new"], inp["q"], cluster_size=cluster_size, kernel=kernel)
     assert case.tree.length == L + C
     kb, vb = bits(inp["k_tok"]), bits(inp["v_tok"])
     kc, vc = O.append_chunk(kb, vb, bits(inp["k_new"]), bits(inp["v_new"]), L)
@@ -221,14 +230,15 @@ def _prefill_check(B, hkv, G, L, C, b, k, cluster_size=0, seed=1):
     (1, 2, 2, 777, 260, 3, 3),     # partial nodes at every level, b = 3
     (1, 1, 8, 250, 20, 16, 8),     # the chunk crosses into a new top level
 ])
-def test_prefill_chunk_matches_oracle(B, hkv, G, L, C, b, k):
-    stats, _ = _prefill_check(B, hkv, G, L, C, b, k)
-    print("prefill", stats)
+@pytest.mark.parametrize("kernel", [0, 1, 2])
+def test_prefill_chunk_matches_oracle(B, hkv, G, L, C, b, k, kernel):
+    stats, _ = _prefill_check(B, hkv, G, L, C, b, k, kernel=kernel)
+    print("prefill", kernel, stats)
 
 
-def test_prefill_cluster_shapes_agree():
-    for cs in (1, 2, 4):
-        _prefill_check(1, 1, 4, 500, 40, 4, 2, cluster_size=cs, seed=9)
+@pytest.mark.parametrize("kernel,cluster_size", SHAPES)
+def test_prefill_launch_shapes(kernel, cluster_size):
+    _prefill_check(1, 1, 4, 500, 40, 4, 2, cluster_size=cluster_size, seed=9, kernel=kernel)
 
 
 def test_prefill_from_empty_cache():
