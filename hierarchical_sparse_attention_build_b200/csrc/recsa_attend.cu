@@ -62,7 +62,9 @@ struct AttendArgs {
   int64_t length;  // decode: L; prefill: L before the chunk
   int64_t row_off[kMaxLevels + 1];
   int64_t slots[kMaxLevels + 1];
-  int64_t span[kMaxLevels + 1];
+  int32_t span[kMaxLevels + 1];   // b^l, saturated above any capacity
+  int32_t nlen[kMaxLevels + 1];   // ceil(length / b^l): nodes of level l at the call's length
+  int32_t levels;                 // levels above the tokens at capacity
   int32_t hkv, hq, b, top_k, nq, causal, out_fp32;
   int32_t sel_levels;
   int32_t table_rows_needed;
@@ -80,36 +82,53 @@ __host__ __device__ constexpr int log2g() {
 
 // ------------------------------------------------------------------ tile geometry
 
+// Per-level geometry, copied to shared memory at kernel start (the level index is a
+// runtime value; shared memory serves it without touching the parameter bank).
+struct Geo {
+  long long row_off[kMaxLevels + 1];
+  long long slots[kMaxLevels + 1];
+  int span[kMaxLevels + 1];
+  int nlen[kMaxLevels + 1];
+};
+constexpr int kGeoBytes = (int)sizeof(Geo);
+
+__device__ __forceinline__ void load_geo(const AttendArgs &a, Geo *g, int tid, int nthreads) {
+  for (int l = tid; l <= kMaxLevels; l += nthreads) {
+    g->row_off[l] = a.row_off[l];
+    g->slots[l] = a.slots[l];
+    g->span[l] = a.span[l];
+    g->nlen[l] = a.nlen[l];
+  }
+}
+
 struct TileInfo {
-  int s, g, qi, T;
-  int64_t p, bh;
+  int s, g, qi, T, p;
+  int64_t bh;
 };
 
-__device__ __forceinline__ TileInfo tile_info(const AttendArgs &a, int tile) {
+__device__ __forceinline__ TileInfo tile_info(const AttendArgs &a, const Geo &geo, int tile) {
   TileInfo t;
   t.qi = tile % a.nq;
   const int sg = tile / a.nq;
   t.g = sg % a.hkv;
   t.s = sg / a.hkv;
-  t.p = a.causal ? a.length + t.qi : a.length;
+  t.p = (int)(a.causal ? a.length + t.qi : a.length);
   t.bh = (int64_t)t.s * a.hkv + t.g;
+  // levels above the tokens: ceil(p / b^T) <= b  <=>  p <= b^(T+1), so T = #{l >= 1 : b^l < p}
   int T = 0;
-  int64_t n = t.p;
-  while (n > a.b) {
-    n = (n + a.b - 1) / a.b;
-    ++T;
-  }
+  while (T < a.levels && geo.span[T + 1] < t.p) ++T;
   t.T = T;
   return t;
 }
 
 // Candidate count of the top level; *forced_pos = position of the forced partial node or -1.
-__device__ __forceinline__ int top_candidates(const AttendArgs &a, const TileInfo &t, int *forced_pos) {
+__device__ __forceinline__ int top_candidates(const AttendArgs &a, const Geo &geo, const TileInfo &t,
+                                              int *forced_pos) {
   *forced_pos = -1;
-  if (t.T == 0) return (int)t.p;
-  if (!a.causal) return (int)((a.length + a.span[t.T] - 1) / a.span[t.T]);
-  const int full = (int)(t.p / a.span[t.T]);
-  if (t.p % a.span[t.T]) {
+  if (t.T == 0) return t.p;
+  if (!a.causal) return geo.nlen[t.T];
+  const int full = t.p / geo.span[t.T];
+  if (t.p - full * geo.span[t.T]) {
     *forced_pos = full;
     return full + 1;
   }
@@ -121,35 +140,33 @@ struct LevelRows {
   int64_t nrows;
 };
 
-__device__ __forceinline__ LevelRows level_rows(const AttendArgs &a, int lvl, int64_t bh) {
+__device__ __forceinline__ LevelRows level_rows(const AttendArgs &a, const Geo &geo, int lvl, int64_t bh) {
   LevelRows r;
   if (lvl == 0) {
     r.k = a.k_tok + bh * a.cap * kD;
     r.v = a.v_tok + bh * a.cap * kD;
     r.nrows = a.cap;
   } else {
-    const int64_t o = (a.row_off[lvl] + bh * a.slots[lvl]) * kD;
+    const int64_t o = (geo.row_off[lvl] + bh * geo.slots[lvl]) * kD;
     r.k = a.k_node + o;
     r.v = a.v_node + o;
-    r.nrows = a.slots[lvl];
+    r.nrows = geo.slots[lvl];
   }
   return r;
 }
 
 // Children of an expanded candidate `v` at level lvl (in node order); *last_forced tells
 // whether the last visible child is itself a partial node (causal mode only).
-__device__ __forceinline__ int child_count(const AttendArgs &a, uint32_t v, int lvl, int64_t p, bool *last_forced) {
-  const int64_t node = v & kNodeMask;
-  const int64_t sb = a.span[lvl - 1];
+__device__ __forceinline__ int child_count(const AttendArgs &a, const Geo &geo, uint32_t v, int lvl, int p,
+                                           bool *last_forced) {
+  const int node = (int)(v & kNodeMask);
   *last_forced = false;
-  if (!a.causal) {
-    const int64_t n_below = (a.length + sb - 1) / sb;
-    return (int)max((int64_t)0, min((int64_t)a.b, n_below - node * a.b));
-  }
+  if (!a.causal) return max(0, min(a.b, geo.nlen[lvl - 1] - node * a.b));
   if (!(v & kForced)) return a.b;
-  const int64_t first = node * a.b;  // children starting before p are visible
-  const int nch = (int)max((int64_t)0, min((int64_t)a.b, (p - first * sb + sb - 1) / sb));
-  if (nch > 0) *last_forced = (first + nch) * sb > p;
+  const int sb = geo.span[lvl - 1];
+  const int first = node * a.b;  // children starting before p are visible
+  const int nch = max(0, min(a.b, (p - first * sb + sb - 1) / sb));
+  if (nch > 0) *last_forced = (int64_t)(first + nch) * sb > p;
   return nch;
 }
 
@@ -220,19 +237,35 @@ __device__ __forceinline__ void rotated_query(const float *qraw, const Trig4 &tq
   }
 }
 
-// Partial dot products of the rotated key row with the G rotated query heads.
+// Partial dot products of the rotated key row with the G rotated query heads
+// (packed fp32 pairs: q2lo[h][u] = (qlo[h][2u], qlo[h][2u+1]), likewise q2hi).
 template <int G>
-__device__ __forceinline__ void dot_row8(const Row8 &k, const Trig4 &tr, const float (&qlo)[G][4],
-                                         const float (&qhi)[G][4], float (&part)[G]) {
+__device__ __forceinline__ void dot_row8(const Row8 &k, const Trig4 &tr, const float2 (&q2lo)[G][2],
+                                         const float2 (&q2hi)[G][2], float (&part)[G]) {
   float lo[4], hi[4];
   unpack_row8(k, lo, hi);
   rotate4(lo, hi, tr);
+  const float2 l01 = make_float2(lo[0], lo[1]), l23 = make_float2(lo[2], lo[3]);
+  const float2 h01 = make_float2(hi[0], hi[1]), h23 = make_float2(hi[2], hi[3]);
 #pragma unroll
   for (int h = 0; h < G; ++h) {
-    float x = 0.f;
+    float2 x = __fmul2_rn(q2lo[h][0], l01);
+    x = __ffma2_rn(q2lo[h][1], l23, x);
+    x = __ffma2_rn(q2hi[h][0], h01, x);
+    x = __ffma2_rn(q2hi[h][1], h23, x);
+    part[h] = x.x + x.y;
+  }
+}
+
+template <int G>
+__device__ __forceinline__ void pack_query(const float (&qlo)[G][4], const float (&qhi)[G][4], float2 (&q2lo)[G][2],
+                                           float2 (&q2hi)[G][2]) {
 #pragma unroll
-    for (int t = 0; t < 4; ++t) x = fmaf(qlo[h][t], lo[t], fmaf(qhi[h][t], hi[t], x));
-    part[h] = x;
+  for (int h = 0; h < G; ++h) {
+    q2lo[h][0] = make_float2(qlo[h][0], qlo[h][1]);
+    q2lo[h][1] = make_float2(qlo[h][2], qlo[h][3]);
+    q2hi[h][0] = make_float2(qhi[h][0], qhi[h][1]);
+    q2hi[h][1] = make_float2(qhi[h][2], qhi[h][3]);
   }
 }
 
@@ -366,14 +399,14 @@ __device__ void warp_write_selection(const AttendArgs &a, const uint32_t *cl, in
 }
 
 // Next level's candidates: the children of the kept and forced candidates, in order.
-__device__ int warp_expand(const AttendArgs &a, const uint32_t *cl, int n, int lvl, int64_t p, uint32_t *nx,
-                           int lane, uint32_t *err) {
+__device__ int warp_expand(const AttendArgs &a, const Geo &geo, const uint32_t *cl, int n, int lvl, int p,
+                           uint32_t *nx, int lane, uint32_t *err) {
   int total = 0;
   for (int base = 0; base < n; base += 32) {
     const int c = base + lane;
     const uint32_t v = c < n ? cl[c] : 0u;
     bool lf = false;
-    const int nch = (c < n && (v & (kKept | kForced))) ? child_count(a, v, lvl, p, &lf) : 0;
+    const int nch = (c < n && (v & (kKept | kForced))) ? child_count(a, geo, v, lvl, p, &lf) : 0;
     int x = nch;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -414,7 +447,7 @@ __device__ __forceinline__ void store_out4(const AttendArgs &a, int64_t at, floa
 // ================================================================== CTA / cluster kernel
 
 struct CtaLayout {
-  int q, cand, skey, slog, red, clm, misc, total;
+  int misc, geo, q, cand, skey, rank, slog, red, clm, total;
 };
 
 __host__ __device__ inline int align128(int x) { return (x + 127) & ~127; }
@@ -427,26 +460,49 @@ __host__ __device__ inline CtaLayout cta_layout(int G, int CS, int max_cand, int
     o = align128(o + bytes);
     return r;
   };
-  L.misc = take(64);
+  L.misc = take(128);
+  L.geo = take(kGeoBytes);
   L.q = take(G * kD * 4);
   L.cand = take(2 * max_cand * 4);
   L.skey = take((CS > 1 ? 2 : 1) * max_cand * 4);
-  L.slog = take(G * own_max * 4);
+  L.rank = take(max_cand * 4);
+  L.slog = take(2 * G * own_max * 4);  // by level parity: the next level scores while this one folds
   L.red = take(kCtaWarps * G * kRedStride * 4);
   L.clm = CS > 1 ? take(CS * G * kRedStride * 4) : 0;
   L.total = o;
   return L;
 }
 
+// Rows a half-warp gathers in one pass of the CTA kernel.
+template <int RPH>
+struct RowSet {
+  Row8 k[RPH], v[RPH];
+  Trig4 tr[RPH];
+  int pos[RPH];
+  bool ok[RPH];
+};
+
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 template <int G, int CS>
 __global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const AttendArgs a) {
+  constexpr int RPH = (CS == 4 || G == 8) ? 2 : 4;  // rows per half-warp per pass (register budget)
+  constexpr int PASS = kHalfWarps * RPH;              // rows per CTA per pass
+  constexpr bool PIPE = RPH == 2;                      // gather the next level before folding this one
   extern __shared__ __align__(128) unsigned char smem[];
   const CtaLayout Ls = cta_layout(G, CS, a.max_cand, a.own_max);
-  int *misc = reinterpret_cast<int *>(smem + Ls.misc);  // [0] next candidate count, [1] workspace bad
+  int *misc = reinterpret_cast<int *>(smem + Ls.misc);  // [1] ws bad, [2..17] warp totals, [24 + parity] next count
+  Geo *geo_s = reinterpret_cast<Geo *>(smem + Ls.geo);
+  load_geo(a, geo_s, threadIdx.x, kCtaThreads);
+  __syncthreads();
+  const Geo &geo = *geo_s;
   float *qraw = reinterpret_cast<float *>(smem + Ls.q);
   uint32_t *cand = reinterpret_cast<uint32_t *>(smem + Ls.cand);
   uint32_t *skey_all = reinterpret_cast<uint32_t *>(smem + Ls.skey);
-  float *slog = reinterpret_cast<float *>(smem + Ls.slog);
+  int *rank = reinterpret_cast<int *>(smem + Ls.rank);
+  float *slog_all = reinterpret_cast<float *>(smem + Ls.slog);
   const int OWN = a.own_max, MC = a.max_cand;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -454,188 +510,337 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const Attend
   int crank = 0;
   if constexpr (CS > 1) crank = (int)cg::this_cluster().block_rank();
   const int tile = blockIdx.x / CS;
-  const TileInfo t = tile_info(a, tile);
+  const TileInfo t = tile_info(a, geo, tile);
   uint32_t *err = &a.hdr->err;
   const int64_t out0 = (((int64_t)t.s * a.nq + t.qi) * a.hq + (int64_t)t.g * G) * kD;
 
-  if (tid == 0) misc[1] = workspace_ok(a) ? 0 : 1;
-  {
-    const uint16_t *qg = a.q + out0;  // q and out share the [B][Q][Hq][128] layout
-    for (int e = tid; e < G * kD / 4; e += kCtaThreads) {
-      const uint2 u = __ldg(reinterpret_cast<const uint2 *>(qg) + e);
-      *reinterpret_cast<float4 *>(qraw + 4 * e) = make_float4(bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y));
-    }
+  // workspace header: read now, checked before the output is written
+  uint32_t hdr_magic = kWsMagic;
+  int hdr_rows = a.table_rows_needed;
+  if (tid == 0) {
+    const volatile WsHeader *h = a.hdr;
+    hdr_magic = h->magic;
+    hdr_rows = h->table_rows;
   }
-  int fpos;
-  int n = top_candidates(a, t, &fpos);
-  for (int i = tid; i < n; i += kCtaThreads) cand[i] = (uint32_t)i | (i == fpos ? kForced : 0u);
-  __syncthreads();
-  if (misc[1]) {  // identical in every CTA of the cluster: leave before any cluster barrier
-    if (tid == 0 && crank == 0) atomicOr(err, kErrWs);
-    if (crank == 0)
-      for (int e = tid; e < G * kD / 4; e += kCtaThreads) store_out4(a, out0 + 4 * e, 0.f, 0.f, 0.f, 0.f);
-    return;
-  }
-  if constexpr (CS > 1) cluster_barrier();  // every peer runs before the first DSMEM store
+  // query rows of the group (q and out share the [B][Q][Hq][128] layout)
+  uint2 qreg = make_uint2(0u, 0u);
+  if (tid < G * kD / 4) qreg = __ldg(reinterpret_cast<const uint2 *>(a.q + out0) + tid);
 
-  float m_w[G], l_w[G], acc[G][8];
+  int fpos;
+  int n = top_candidates(a, geo, t, &fpos);
+  if (n > a.table_rows_needed - 1) {  // cannot happen for a valid launch; guards the table reads
+    if (tid == 0) atomicOr(err, kErrCount);
+    n = a.table_rows_needed - 1;
+  }
+
+  // Gather rows [pass0, pass0 + PASS) of this CTA's slice [.., hi_r) of level lvl.  cl == nullptr
+  // means the top level, whose position i is node i.
+  auto gather = [&](RowSet<RPH> &rs, int lvl, const uint32_t *cl, int pass0, int hi_r, bool values) {
+    const LevelRows lr = level_rows(a, geo, lvl, t.bh);
+#pragma unroll
+    for (int r = 0; r < RPH; ++r) {
+      const int i = pass0 + hw + kHalfWarps * r;
+      rs.pos[r] = i;
+      const uint32_t c = i < hi_r ? (cl ? cl[i] : ((uint32_t)i | (i == fpos ? kForced : 0u))) : kForced;
+      const int64_t node = c & kNodeMask;
+      rs.ok[r] = i < hi_r && !(c & kForced) && node < lr.nrows;
+      if (i < hi_r && !(c & kForced) && node >= lr.nrows && j16 == 0) atomicOr(err, kErrIndex);
+      if (rs.ok[r]) {
+        rs.k[r] = ldg_row8(lr.k + node * kD, j16);
+        rs.tr[r] = ldg_trig4(a.table, i, j16);
+        if (values) rs.v[r] = ldg_row8(lr.v + node * kD, j16);
+      }
+    }
+  };
+
+  float m_w[G], l_w[G];
+  float2 acc[G][4];  // dims (4j, 4j+1), (4j+2, 4j+3), (64+4j, ..), (64+4j+2, ..)
 #pragma unroll
   for (int h = 0; h < G; ++h) {
     m_w[h] = -INFINITY;
     l_w[h] = 0.f;
 #pragma unroll
-    for (int d = 0; d < 8; ++d) acc[h][d] = 0.f;
+    for (int d = 0; d < 4; ++d) acc[h][d] = make_float2(0.f, 0.f);
   }
-  int cur = 0, keys_read = 0, values_read = 0;
 
-  // Fold up to two rows per half-warp (values in registers) into the warp's state.
-  auto fold_rows = [&](const Row8 (&vr)[2], const int (&ii)[2], const bool (&ent)[2], int lo_r) {
+  // Fold the entry rows of a row set (values in registers) into the warp's state.
+  auto fold = [&](const RowSet<RPH> &rs, const bool (&ent)[RPH], const float *slog, int lo_r) {
     float mx[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) mx[h] = -INFINITY;
 #pragma unroll
-    for (int r = 0; r < 2; ++r)
+    for (int r = 0; r < RPH; ++r)
       if (ent[r]) {
 #pragma unroll
-        for (int h = 0; h < G; ++h) mx[h] = fmaxf(mx[h], slog[h * OWN + ii[r] - lo_r]);
+        for (int h = 0; h < G; ++h) mx[h] = fmaxf(mx[h], slog[h * OWN + rs.pos[r] - lo_r]);
       }
-    float mnew[G], alpha[G];
+    float mnew[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 16));
       mnew[h] = fmaxf(m_w[h], mx[h]);
-      alpha[h] = (mnew[h] == -INFINITY) ? 1.f : expf(m_w[h] - mnew[h]);
+      const float alpha = (mnew[h] == -INFINITY) ? 1.f : __expf(m_w[h] - mnew[h]);
       m_w[h] = mnew[h];
-      l_w[h] *= alpha[h];
+      l_w[h] *= alpha;
+      const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-      for (int d = 0; d < 8; ++d) acc[h][d] *= alpha[h];
+      for (int d = 0; d < 4; ++d) acc[h][d] = __fmul2_rn(acc[h][d], a2);
     }
     float ls[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) ls[h] = 0.f;
 #pragma unroll
-    for (int r = 0; r < 2; ++r)
+    for (int r = 0; r < RPH; ++r)
       if (ent[r]) {
-        float lo[4], hi[4];
-        unpack_row8(vr[r], lo, hi);
+        const Row8 &v = rs.v[r];
+        const float2 v0 = make_float2(bf16_lo(v.lo.x), bf16_hi(v.lo.x)), v1 = make_float2(bf16_lo(v.lo.y), bf16_hi(v.lo.y));
+        const float2 v2 = make_float2(bf16_lo(v.hi.x), bf16_hi(v.hi.x)), v3 = make_float2(bf16_lo(v.hi.y), bf16_hi(v.hi.y));
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          const float pr = expf(slog[h * OWN + ii[r] - lo_r] - mnew[h]);
+          const float pr = __expf(slog[h * OWN + rs.pos[r] - lo_r] - mnew[h]);
           ls[h] += pr;
-#pragma unroll
-          for (int d = 0; d < 4; ++d) {
-            acc[h][d] = fmaf(pr, lo[d], acc[h][d]);
-            acc[h][4 + d] = fmaf(pr, hi[d], acc[h][4 + d]);
-          }
+          const float2 p2 = make_float2(pr, pr);
+          acc[h][0] = __ffma2_rn(p2, v0, acc[h][0]);
+          acc[h][1] = __ffma2_rn(p2, v1, acc[h][1]);
+          acc[h][2] = __ffma2_rn(p2, v2, acc[h][2]);
+          acc[h][3] = __ffma2_rn(p2, v3, acc[h][3]);
         }
       }
 #pragma unroll
     for (int h = 0; h < G; ++h) l_w[h] += ls[h] + __shfl_xor_sync(0xffffffffu, ls[h], 16);
   };
 
+  // the top level's rows go out before anything waits on memory
+  int per = (n + CS - 1) / CS;
+  int lo_r = min(n, crank * per), hi_r = min(n, lo_r + per);
+  RowSet<RPH> cur_rs, nxt_rs;
+  bool preloaded = false;
+  Trig4 tq_pre;
+  if (hi_r - lo_r <= PASS) {
+    gather(cur_rs, t.T, nullptr, lo_r, hi_r, true);
+    tq_pre = ldg_trig4(a.table, n, j16);
+    preloaded = true;
+  }
+  if (tid < G * kD / 4)
+    *reinterpret_cast<float4 *>(qraw + 4 * tid) =
+        make_float4(bf16_lo(qreg.x), bf16_hi(qreg.x), bf16_lo(qreg.y), bf16_hi(qreg.y));
+  for (int i = tid; i < n; i += kCtaThreads) {
+    cand[i] = (uint32_t)i | (i == fpos ? kForced : 0u);
+    rank[i] = 0;
+  }
+  if (tid == 0) misc[1] = (hdr_magic != kWsMagic || hdr_rows < a.table_rows_needed) ? 1 : 0;
+  __syncthreads();
+  if constexpr (CS > 1) cluster_barrier();  // every peer runs before the first DSMEM store
+
+  int cur = 0, keys_read = 0, values_read = 0;
   for (int lvl = t.T; lvl >= 0; --lvl) {
     uint32_t *cl = cand + cur * MC;
     uint32_t *sk = skey_all + ((CS > 1) ? (lvl & 1) * MC : 0);
-    if (n > a.table_rows_needed - 1) {  // cannot happen for a valid launch; guards the table read
-      if (tid == 0) atomicOr(err, kErrCount);
-      n = a.table_rows_needed - 1;
-    }
-    const int per = (n + CS - 1) / CS;
-    const int lo_r = min(n, crank * per);
-    const int hi_r = min(n, lo_r + per);
-    const bool single = hi_r - lo_r <= kPassRows;
-    const LevelRows lr = level_rows(a, lvl, t.bh);
-    const Trig4 tq = ldg_trig4(a.table, n, j16);
+    float *slog = slog_all + (lvl & 1) * G * OWN;
+    const bool single = hi_r - lo_r <= PASS;
+    const LevelRows lr = level_rows(a, geo, lvl, t.bh);
 
-    // 1. gather and score this CTA's slice; in one pass the values come along
-    Row8 vr[2];
-    int ii[2] = {lo_r, lo_r};
-    bool ent[2] = {false, false};
-    for (int pass0 = lo_r; pass0 < hi_r; pass0 += kPassRows) {
-      Row8 kr[2];
-      Trig4 tr[2];
-      bool ok[2];
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int i = pass0 + hw + kHalfWarps * r;
-        ii[r] = i;
-        const uint32_t c = i < hi_r ? cl[i] : kForced;
-        const int64_t node = c & kNodeMask;
-        ok[r] = i < hi_r && !(c & kForced) && node < lr.nrows;
-        if (i < hi_r && !(c & kForced) && node >= lr.nrows && j16 == 0) atomicOr(err, kErrIndex);
-        if (ok[r]) {
-          kr[r] = ldg_row8(lr.k + node * kD, j16);
-          tr[r] = ldg_trig4(a.table, i, j16);
-          if (single) vr[r] = ldg_row8(lr.v + node * kD, j16);
-        }
-      }
+    // 1. score this CTA's slice (rows preloaded, or gathered now)
+    const Trig4 tq = preloaded ? tq_pre : ldg_trig4(a.table, n, j16);
+    if (single && !preloaded) gather(cur_rs, lvl, cl, lo_r, hi_r, true);
+    float2 q2lo[G][2], q2hi[G][2];
+    {
       float qlo[G][4], qhi[G][4];
       rotated_query<G>(qraw, tq, j16, qlo, qhi);
+      pack_query<G>(qlo, qhi, q2lo, q2hi);
+    }
+    auto score = [&](const RowSet<RPH> &rs) {
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
+      for (int r = 0; r < RPH; ++r) {
         float part[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) part[h] = 0.f;
-        if (ok[r]) dot_row8<G>(kr[r], tr[r], qlo, qhi, part);
+        if (rs.ok[r]) dot_row8<G>(rs.k[r], rs.tr[r], q2lo, q2hi, part);
         const float x = reduce16<G>(part, j16) * a.scale;
         const float S = group_sum16<G>(x);
-        if (ok[r]) {
-          if (head_writer<G>(j16)) slog[head_of<G>(j16) * OWN + ii[r] - lo_r] = x;
+        if (rs.ok[r]) {
+          if (head_writer<G>(j16)) slog[head_of<G>(j16) * OWN + rs.pos[r] - lo_r] = x;
           if (lvl > 0 && j16 == 0) {
             const uint32_t key = order_key(S);
             if constexpr (CS > 1) {
               cg::cluster_group cluster = cg::this_cluster();
 #pragma unroll
-              for (int q = 0; q < CS; ++q) cluster.map_shared_rank(sk, q)[ii[r]] = key;
+              for (int q = 0; q < CS; ++q) cluster.map_shared_rank(sk, q)[rs.pos[r]] = key;
             } else {
-              sk[ii[r]] = key;
+              sk[rs.pos[r]] = key;
             }
           }
         }
-        ent[r] = ok[r];
+      }
+    };
+    if (single) {
+      score(cur_rs);
+    } else {
+      for (int pass0 = lo_r; pass0 < hi_r; pass0 += PASS) {
+        RowSet<RPH> rs;
+        gather(rs, lvl, cl, pass0, hi_r, false);
+        score(rs);
       }
     }
-    int nforced = (a.causal && n > 0 && (cl[n - 1] & kForced)) ? 1 : 0;
+    preloaded = false;
+    // the next count slot of this level's parity was last read two levels ago
+    int *next_count = misc + 24 + (lvl & 1);
+    if (tid == 0) *next_count = 0;
+    const int nforced = (a.causal && n > 0 && (cl[n - 1] & kForced)) ? 1 : 0;
     const int m = n - nforced;
     keys_read += m;
     if constexpr (CS > 1) cluster_barrier();
     __syncthreads();
 
-    // 2. selection (one warp), then fold own entries while that warp expands
+    int n_next = 0;
     if (lvl > 0) {
-      if (warp == 0) {
-        warp_topk(cl, sk, n, a.top_k, lane);
-        if (crank == 0) warp_write_selection(a, cl, n, lvl, tile, lane);
+      // 2. top-k by rank: a candidate is kept when fewer than k scorable candidates beat it
+      const bool keep_all = a.top_k >= m;
+      if (!keep_all && a.top_k > 0) {
+        // items (candidate c, 64-wide segment of competitors); the forced candidate, if
+        // any, is the last one and competes with nobody (c < m)
+        const int nseg = (m + 63) / 64;
+        for (int it = tid; it < m * nseg; it += kCtaThreads) {
+          const int seg = it / m, c = it - seg * m;
+          const uint32_t kc = sk[c];
+          const int e0 = seg * 64, e1 = min(m, e0 + 64);
+          const int mid = max(e0, min(c, e1));  // competitors below c win ties
+          int better = 0;
+          int e = e0;
+          for (; e + 4 <= mid; e += 4) {
+            const uint4 k4 = *reinterpret_cast<const uint4 *>(sk + e);
+            better += (k4.x >= kc) + (k4.y >= kc) + (k4.z >= kc) + (k4.w >= kc);
+          }
+          for (; e < mid; ++e) better += sk[e] >= kc;
+          if (e == c) ++e;
+          for (; e < e1 && (e & 3); ++e) better += sk[e] > kc;
+          for (; e + 4 <= e1; e += 4) {
+            const uint4 k4 = *reinterpret_cast<const uint4 *>(sk + e);
+            better += (k4.x > kc) + (k4.y > kc) + (k4.z > kc) + (k4.w > kc);
+          }
+          for (; e < e1; ++e) better += sk[e] > kc;
+          if (better) atomicAdd(&rank[c], better);
+        }
+        __syncthreads();
       }
-      __syncthreads();
       values_read += m - min(a.top_k, m);
+      // 3. kept flags and the next candidate list.  Expanded candidates (kept, or forced)
+      //    are in node order and all but the last have exactly b children, so the e-th
+      //    expanded candidate's children start at position e * b.
+      uint32_t *nx = cand + (cur ^ 1) * MC;
+      const LevelRows lb = level_rows(a, geo, lvl - 1, t.bh);
+      int carry_e = 0, carry_k = 0;
+      int32_t *sel = (a.sel_idx != nullptr && crank == 0 && lvl <= a.sel_levels)
+                         ? a.sel_idx + ((int64_t)tile * a.sel_levels + (lvl - 1)) * a.top_k
+                         : nullptr;
+      for (int base = 0; base < n; base += kCtaThreads) {
+        const int c = base + tid;
+        const uint32_t v = c < n ? cl[c] : 0u;
+        const bool forced = c < n && (v & kForced);
+        const bool kept = c < n && !forced && a.top_k > 0 && (keep_all || rank[c] < a.top_k);
+        const bool ex = kept || forced;
+        const unsigned be = __ballot_sync(0xffffffffu, ex), bk = __ballot_sync(0xffffffffu, kept);
+        if (lane == 0) {
+          misc[2 + warp] = __popc(be);
+          misc[2 + kCtaWarps + warp] = __popc(bk);
+        }
+        __syncthreads();
+        int pe = carry_e + __popc(be & ((1u << lane) - 1u)), pk = carry_k + __popc(bk & ((1u << lane) - 1u));
+        int te = 0, tk = 0;
+#pragma unroll
+        for (int w = 0; w < kCtaWarps; ++w) {
+          const int xe = misc[2 + w], xk = misc[2 + kCtaWarps + w];
+          if (w < warp) {
+            pe += xe;
+            pk += xk;
+          }
+          te += xe;
+          tk += xk;
+        }
+        if (kept) {
+          cl[c] = v | kKept;
+          if (sel && pk < a.top_k) sel[pk] = (int32_t)(v & kNodeMask);
+        }
+        if (ex) {
+          bool lf = false;
+          const int nch = child_count(a, geo, v, lvl, t.p, &lf);
+          const int off = pe * a.b;
+          const int64_t first = (int64_t)(v & kNodeMask) * a.b;
+          for (int u = 0; u < nch; ++u) {
+            if (off + u >= MC) {
+              atomicOr(err, kErrCount);
+              break;
+            }
+            nx[off + u] = (uint32_t)(first + u) | ((lf && u == nch - 1) ? kForced : 0u);
+          }
+          atomicMax(next_count, off + nch);
+          // warm L2 with the rows the next level gathers (one CTA of the cluster per node)
+          if (nch > 0 && pe % CS == crank && first + nch <= lb.nrows) {
+            prefetch_l2(lb.k + first * kD, (uint32_t)nch * kRowBytes);
+            prefetch_l2(lb.v + first * kD, (uint32_t)nch * kRowBytes);
+          }
+        }
+        __syncthreads();
+        carry_e += te;
+        carry_k += tk;
+      }
+      if (sel)
+        for (int u = carry_k + tid; u < a.top_k; u += kCtaThreads) sel[u] = -1;
+      n_next = min(*next_count, MC);
+      if (n_next > a.table_rows_needed - 1) {
+        if (tid == 0) atomicOr(err, kErrCount);
+        n_next = a.table_rows_needed - 1;
+      }
+      for (int i = tid; i < n_next; i += kCtaThreads) rank[i] = 0;  // for the next level's count
     } else {
       values_read += n;
     }
-    if (lvl > 0 && warp == 0) misc[0] = warp_expand(a, cl, n, lvl, t.p, cand + (cur ^ 1) * MC, lane, err);
+
+    // 4. next level's rows go out before this level's fold (the pipelined shape)
+    const int per2 = (n_next + CS - 1) / CS;
+    const int lo2 = min(n_next, crank * per2), hi2 = min(n_next, lo2 + per2);
+    if (PIPE && lvl > 0 && hi2 - lo2 <= PASS) {
+      gather(nxt_rs, lvl - 1, cand + (cur ^ 1) * MC, lo2, hi2, true);
+      tq_pre = ldg_trig4(a.table, n_next, j16);
+      preloaded = true;
+    }
+    // 5. fold this level's entries
     if (single) {
-      if (lvl > 0) {
+      bool ent[RPH];
 #pragma unroll
-        for (int r = 0; r < 2; ++r) ent[r] = ent[r] && !(cl[ii[r]] & kKept);
-      }
-      fold_rows(vr, ii, ent, lo_r);
+      for (int r = 0; r < RPH; ++r) ent[r] = cur_rs.ok[r] && (lvl == 0 || !(cl[cur_rs.pos[r]] & kKept));
+      fold(cur_rs, ent, slog, lo_r);
     } else {
-      for (int pass0 = lo_r; pass0 < hi_r; pass0 += kPassRows) {
+      for (int pass0 = lo_r; pass0 < hi_r; pass0 += PASS) {
+        RowSet<RPH> rs;
+        bool ent[RPH];
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
+        for (int r = 0; r < RPH; ++r) {
           const int i = pass0 + hw + kHalfWarps * r;
-          ii[r] = i;
+          rs.pos[r] = i;
           const uint32_t c = i < hi_r ? cl[i] : (kForced | kKept);
           const int64_t node = c & kNodeMask;
           ent[r] = i < hi_r && !(c & (kForced | kKept)) && node < lr.nrows;
-          if (ent[r]) vr[r] = ldg_row8(lr.v + node * kD, j16);
+          rs.ok[r] = ent[r];
+          if (ent[r]) rs.v[r] = ldg_row8(lr.v + node * kD, j16);
         }
-        fold_rows(vr, ii, ent, lo_r);
+        fold(rs, ent, slog, lo_r);
       }
     }
     if (lvl == 0) break;
-    __syncthreads();
-    n = misc[0];
+    if (preloaded) {
+#pragma unroll
+      for (int r = 0; r < RPH; ++r) {
+        cur_rs.k[r] = nxt_rs.k[r];
+        cur_rs.v[r] = nxt_rs.v[r];
+        cur_rs.tr[r] = nxt_rs.tr[r];
+        cur_rs.pos[r] = nxt_rs.pos[r];
+        cur_rs.ok[r] = nxt_rs.ok[r];
+      }
+    }
+    n = n_next;
+    lo_r = lo2;
+    hi_r = hi2;
     cur ^= 1;
   }
 
@@ -648,19 +853,24 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const Attend
   float *red = reinterpret_cast<float *>(smem + Ls.red);  // [warp][h][kRedStride]: m, l, pad, acc[128]
 #pragma unroll
   for (int h = 0; h < G; ++h) {
+    float2 x[4];
 #pragma unroll
-    for (int d = 0; d < 8; ++d) acc[h][d] += __shfl_xor_sync(0xffffffffu, acc[h][d], 16);
+    for (int d = 0; d < 4; ++d) {
+      x[d].x = acc[h][d].x + __shfl_xor_sync(0xffffffffu, acc[h][d].x, 16);
+      x[d].y = acc[h][d].y + __shfl_xor_sync(0xffffffffu, acc[h][d].y, 16);
+    }
     float *r = red + (warp * G + h) * kRedStride;
     if (lane == 0) {
       r[0] = m_w[h];
       r[1] = l_w[h];
     }
     if (lane < 16) {
-      *reinterpret_cast<float4 *>(r + 4 + 4 * j16) = make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
-      *reinterpret_cast<float4 *>(r + 4 + kHalf + 4 * j16) = make_float4(acc[h][4], acc[h][5], acc[h][6], acc[h][7]);
+      *reinterpret_cast<float4 *>(r + 4 + 4 * j16) = make_float4(x[0].x, x[0].y, x[1].x, x[1].y);
+      *reinterpret_cast<float4 *>(r + 4 + kHalf + 4 * j16) = make_float4(x[2].x, x[2].y, x[3].x, x[3].y);
     }
   }
   __syncthreads();
+  const bool ws_bad = misc[1] != 0;
   float *clm = reinterpret_cast<float *>(smem + Ls.clm);  // [rank][h][kRedStride] on cluster rank 0
   for (int e = tid; e < G * kD / 4; e += kCtaThreads) {
     const int h = (4 * e) / kD, d0 = (4 * e) % kD;
@@ -672,14 +882,14 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const Attend
 #pragma unroll
       for (int w = 0; w < kCtaWarps; ++w) {
         const float *r = red + (w * G + h) * kRedStride;
-        const float f = (r[0] == -INFINITY) ? 0.f : expf(r[0] - M);
+        const float f = (r[0] == -INFINITY) ? 0.f : __expf(r[0] - M);
         l += f * r[1];
 #pragma unroll
         for (int d = 0; d < 4; ++d) o[d] += f * r[4 + d0 + d];
       }
     }
     if constexpr (CS == 1) {
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float inv = (l > 0.f && !ws_bad) ? 1.f / l : 0.f;
       store_out4(a, out0 + 4 * e, o[0] * inv, o[1] * inv, o[2] * inv, o[3] * inv);
     } else {
       cg::cluster_group cluster = cg::this_cluster();
@@ -705,17 +915,18 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const Attend
 #pragma unroll
           for (int r = 0; r < CS; ++r) {
             const float *x = clm + (r * G + h) * kRedStride;
-            const float f = (x[0] == -INFINITY) ? 0.f : expf(x[0] - M);
+            const float f = (x[0] == -INFINITY) ? 0.f : __expf(x[0] - M);
             l += f * x[1];
 #pragma unroll
             for (int d = 0; d < 4; ++d) o[d] += f * x[4 + d0 + d];
           }
         }
-        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const float inv = (l > 0.f && !ws_bad) ? 1.f / l : 0.f;
         store_out4(a, out0 + 4 * e, o[0] * inv, o[1] * inv, o[2] * inv, o[3] * inv);
       }
     }
   }
+  if (ws_bad && tid == 0 && crank == 0) atomicOr(err, kErrWs);
 }
 
 // ================================================================== warp-per-tile kernel
@@ -739,9 +950,13 @@ __global__ void __launch_bounds__(kWarpKernelMaxWarps * 32, (G <= 4 ? 2 : 1)) at
   const bool ws_ok = workspace_ok(a);
   if (!ws_ok && threadIdx.x == 0 && blockIdx.x == 0) atomicOr(err, kErrWs);
   const int nw = gridDim.x * a.warps_per_block;
+  Geo *geo_s = reinterpret_cast<Geo *>(smem + (size_t)a.warps_per_block * warp_slice_bytes(G, MC));
+  load_geo(a, geo_s, threadIdx.x, blockDim.x);
+  __syncthreads();
+  const Geo &geo = *geo_s;
 
   for (int tile = blockIdx.x * a.warps_per_block + wib; tile < a.tiles; tile += nw) {
-    const TileInfo t = tile_info(a, tile);
+    const TileInfo t = tile_info(a, geo, tile);
     const int64_t out0 = (((int64_t)t.s * a.nq + t.qi) * a.hq + (int64_t)t.g * G) * kD;
     if (!ws_ok) {
 #pragma unroll
@@ -755,17 +970,17 @@ __global__ void __launch_bounds__(kWarpKernelMaxWarps * 32, (G <= 4 ? 2 : 1)) at
           make_float4(bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y));
     }
     int fpos;
-    int n = top_candidates(a, t, &fpos);
+    int n = top_candidates(a, geo, t, &fpos);
     for (int i = lane; i < n; i += 32) cand[i] = (uint32_t)i | (i == fpos ? kForced : 0u);
     __syncwarp();
 
-    float m_w[G], l_w[G], acc[G][4];
+    float m_w[G], l_w[G];
+    float2 acc[G][2];  // dims (4 lane, 4 lane + 1), (4 lane + 2, 4 lane + 3)
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       m_w[h] = -INFINITY;
       l_w[h] = 0.f;
-#pragma unroll
-      for (int d = 0; d < 4; ++d) acc[h][d] = 0.f;
+      acc[h][0] = acc[h][1] = make_float2(0.f, 0.f);
     }
     int cur = 0, keys_read = 0, values_read = 0;
 
@@ -775,9 +990,13 @@ __global__ void __launch_bounds__(kWarpKernelMaxWarps * 32, (G <= 4 ? 2 : 1)) at
         if (lane == 0) atomicOr(err, kErrCount);
         n = a.table_rows_needed - 1;
       }
-      const LevelRows lr = level_rows(a, lvl, t.bh);
-      float qlo[G][4], qhi[G][4];
-      rotated_query<G>(qraw, ldg_trig4(a.table, n, j16), j16, qlo, qhi);
+      const LevelRows lr = level_rows(a, geo, lvl, t.bh);
+      float2 q2lo[G][2], q2hi[G][2];
+      {
+        float qlo[G][4], qhi[G][4];
+        rotated_query<G>(qraw, ldg_trig4(a.table, n, j16), j16, qlo, qhi);
+        pack_query<G>(qlo, qhi, q2lo, q2hi);
+      }
 
       // keys pass: one row per half-warp per step, the next step's loads in flight
       Row8 kr_n;
@@ -803,11 +1022,11 @@ __global__ void __launch_bounds__(kWarpKernelMaxWarps * 32, (G <= 4 ? 2 : 1)) at
         float part[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) part[h] = 0.f;
-        if (ok) dot_row8<G>(kr, tr, qlo, qhi, part);
+        if (ok) dot_row8<G>(kr, tr, q2lo, q2hi, part);
         const float x = reduce16<G>(part, j16) * a.scale;
         const float S = group_sum16<G>(x);
         if (ok) {
-          if (head_writer<G>(j16)) slog[head_of<G>(j16) * MC + i] = x;
+          if (head_writer<G>(j16)) slog[i * G + head_of<G>(j16)] = x;
           if (j16 == 0) skey[i] = order_key(S);
         }
       }
@@ -842,18 +1061,19 @@ __global__ void __launch_bounds__(kWarpKernelMaxWarps * 32, (G <= 4 ? 2 : 1)) at
       for (int e = lane; e < ne; e += 32) {
         const int pos = list[e];
 #pragma unroll
-        for (int h = 0; h < G; ++h) mx[h] = fmaxf(mx[h], slog[h * MC + pos]);
+        for (int h = 0; h < G; ++h) mx[h] = fmaxf(mx[h], slog[pos * G + h]);
       }
       float mnew[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         mx[h] = warp_max(mx[h]);
         mnew[h] = fmaxf(m_w[h], mx[h]);
-        const float alpha = (mnew[h] == -INFINITY) ? 1.f : expf(m_w[h] - mnew[h]);
+        const float alpha = (mnew[h] == -INFINITY) ? 1.f : __expf(m_w[h] - mnew[h]);
         m_w[h] = mnew[h];
         l_w[h] *= alpha;
-#pragma unroll
-        for (int d = 0; d < 4; ++d) acc[h][d] *= alpha;
+        const float2 a2 = make_float2(alpha, alpha);
+        acc[h][0] = __fmul2_rn(acc[h][0], a2);
+        acc[h][1] = __fmul2_rn(acc[h][1], a2);
       }
       float ls[G];
 #pragma unroll
@@ -862,8 +1082,8 @@ __global__ void __launch_bounds__(kWarpKernelMaxWarps * 32, (G <= 4 ? 2 : 1)) at
         const int pos = list[e];
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          const float pr = expf(slog[h * MC + pos] - mnew[h]);
-          slog[h * MC + pos] = pr;
+          const float pr = __expf(slog[pos * G + h] - mnew[h]);
+          slog[pos * G + h] = pr;
           ls[h] += pr;
         }
       }
@@ -882,19 +1102,32 @@ __global__ void __launch_bounds__(kWarpKernelMaxWarps * 32, (G <= 4 ? 2 : 1)) at
         for (int u = 0; u < 8; ++u)
           if (e0 + u < ne) {
             const int pos = list[e0 + u];
-            const float v0 = bf16_lo(vv[u].x), v1 = bf16_hi(vv[u].x), v2 = bf16_lo(vv[u].y), v3 = bf16_hi(vv[u].y);
+            const float2 v01 = make_float2(bf16_lo(vv[u].x), bf16_hi(vv[u].x));
+            const float2 v23 = make_float2(bf16_lo(vv[u].y), bf16_hi(vv[u].y));
+            float pr[G];
+            if constexpr (G % 4 == 0) {
+#pragma unroll
+              for (int h4 = 0; h4 < G; h4 += 4) {
+                const float4 p4 = *reinterpret_cast<const float4 *>(slog + pos * G + h4);
+                pr[h4] = p4.x;
+                pr[h4 + 1] = p4.y;
+                pr[h4 + 2] = p4.z;
+                pr[h4 + 3] = p4.w;
+              }
+            } else {
+#pragma unroll
+              for (int h = 0; h < G; ++h) pr[h] = slog[pos * G + h];
+            }
 #pragma unroll
             for (int h = 0; h < G; ++h) {
-              const float pr = slog[h * MC + pos];
-              acc[h][0] = fmaf(pr, v0, acc[h][0]);
-              acc[h][1] = fmaf(pr, v1, acc[h][1]);
-              acc[h][2] = fmaf(pr, v2, acc[h][2]);
-              acc[h][3] = fmaf(pr, v3, acc[h][3]);
+              const float2 p2 = make_float2(pr[h], pr[h]);
+              acc[h][0] = __ffma2_rn(p2, v01, acc[h][0]);
+              acc[h][1] = __ffma2_rn(p2, v23, acc[h][1]);
             }
           }
       }
       if (lvl == 0) break;
-      n = warp_expand(a, cl, n, lvl, t.p, cand + (cur ^ 1) * MC, lane, err);
+      n = warp_expand(a, geo, cl, n, lvl, t.p, cand + (cur ^ 1) * MC, lane, err);
       cur ^= 1;
       __syncwarp();
     }
@@ -902,7 +1135,8 @@ __global__ void __launch_bounds__(kWarpKernelMaxWarps * 32, (G <= 4 ? 2 : 1)) at
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       const float inv = l_w[h] > 0.f ? 1.f / l_w[h] : 0.f;
-      store_out4(a, out0 + h * kD + 4 * lane, acc[h][0] * inv, acc[h][1] * inv, acc[h][2] * inv, acc[h][3] * inv);
+      store_out4(a, out0 + h * kD + 4 * lane, acc[h][0].x * inv, acc[h][0].y * inv, acc[h][1].x * inv,
+                 acc[h][1].y * inv);
     }
     if (a.entries != nullptr && lane == 0) {
       a.entries[2 * (int64_t)tile] = keys_read;
@@ -960,7 +1194,7 @@ int launch_warp(const AttendArgs &args, cudaStream_t stream) {
   AttendArgs a = args;
   const int slice = warp_slice_bytes(G, a.max_cand);
   const int sms = sm_count_cached();
-  int wpb = std::min(kWarpKernelMaxWarps, (227 * 1024) / slice);
+  int wpb = std::min(kWarpKernelMaxWarps, (227 * 1024 - kGeoBytes) / slice);
   // few tiles: spread them over the SMs rather than packing 8 per CTA
   wpb = std::max(1, std::min(wpb, (a.tiles + sms - 1) / sms));
   if (wpb < 1) {
@@ -968,7 +1202,7 @@ int launch_warp(const AttendArgs &args, cudaStream_t stream) {
     return -1;
   }
   a.warps_per_block = wpb;
-  const int smem = wpb * slice;
+  const int smem = wpb * slice + kGeoBytes;
   auto kern = attend_warp_kernel<G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return (int)e;
@@ -1013,8 +1247,11 @@ int launch_attend(const AttendLaunch &l, void *stream) {
   for (int i = 0; i <= kMaxLevels; ++i) {
     a.row_off[i] = l.geom.row_off[i];
     a.slots[i] = l.geom.slots[i];
-    a.span[i] = l.geom.span[i];
+    const int64_t sp = std::min<int64_t>(l.geom.span[i], (int64_t)1 << 30 | 1);
+    a.span[i] = (int32_t)sp;
+    a.nlen[i] = (int32_t)((l.length + sp - 1) / sp);
   }
+  a.levels = l.geom.levels_cap;
   a.hkv = l.geom.hkv;
   a.hq = l.geom.hkv * l.group;
   a.b = l.geom.b;
@@ -1028,7 +1265,7 @@ int launch_attend(const AttendLaunch &l, void *stream) {
   a.tiles = l.geom.batch * l.geom.hkv * l.num_queries;
   const int sms = sm_count_cached();
   int kernel = l.kernel;
-  if (kernel == 0) kernel = (a.tiles <= 2 * sms) ? 1 : 2;  // CTA per tile while it fits two waves
+  if (kernel == 0) kernel = (a.tiles <= sms) ? 1 : 2;  // CTA per tile while every tile has its own SM
   int CS = l.cluster_size;
   if (kernel == 1 && CS == 0) CS = (a.tiles * 4 <= sms) ? 4 : (a.tiles * 2 <= sms) ? 2 : 1;
   int rc;
