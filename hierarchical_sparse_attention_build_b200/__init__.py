@@ -96,6 +96,7 @@ def _load() -> ctypes.CDLL:
         "recsa_decode": [P, T, vp, i32, vp, i32, vp, sz, D, vp],
         "recsa_prefill_chunk": [P, T, vp, vp, vp, i32, vp, i32, vp, sz, D, vp],
         "recsa_check_device_errors": [vp, vp],
+        "recsa_decode_no_alloc": [P, T, vp, i32, vp, i32, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -237,6 +238,13 @@ def prefill_chunk(p: Params, tree: RecsaTree, k_new: torch.Tensor, v_new: torch.
     _check(_lib.recsa_prefill_chunk(ctypes.byref(p), ctypes.byref(tree.c), _ptr(k_new), _ptr(v_new), _ptr(q), chunk,
                                     _ptr(out), int(out.dtype == torch.float32), _ptr(ws.buf), ws.nbytes,
                                     ctypes.byref(dbg) if dbg is not None else None, _stream(stream)))
+
+
+def decode_no_alloc(p: Params, tree: RecsaTree, q: torch.Tensor, out: torch.Tensor, stream=None) -> None:
+    """recsa_decode_no_alloc: recsa_decode with its scratch in the library's fixed device array."""
+    assert q.dtype == torch.bfloat16 and q.is_contiguous() and out.is_contiguous()
+    _check(_lib.recsa_decode_no_alloc(ctypes.byref(p), ctypes.byref(tree.c), _ptr(q), q.shape[1], _ptr(out),
+                                      int(out.dtype == torch.float32), _stream(stream)))
 
 
 def check_device_errors(ws: Workspace, stream=None) -> None:

@@ -14,7 +14,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "librecsa.so")
 OBJ_DIR = os.path.join(PKG, "_build")
 
-SOURCES = ["recsa_abi.cpp", "recsa_build.cu", "recsa_attend.cu"]
+SOURCES = ["recsa_abi.cpp", "recsa_build.cu", "recsa_attend.cu", "recsa_no_alloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden", "-I", INCLUDE, "-I", CSRC]
 

@@ -182,6 +182,27 @@ RECSA_API recsa_status recsa_prefill_chunk(const recsa_params *params, recsa_tre
                                            int32_t out_is_fp32, void *ws, size_t ws_bytes,
                                            const recsa_debug *debug, recsa_stream_t stream);
 
+/* Decode without any device allocation.  The RecSA paper has no counterpart to this
+ * call; it exists for callers that cannot allocate device memory for a workspace:
+ * hosts that give the library a fixed memory budget and own every allocation, serving
+ * loops that forbid allocation after warm-up, or code that must not touch the
+ * allocator while other work holds it.  Same inputs, outputs and results as
+ * recsa_decode (no debug outputs); the RoPE table and error word live in a fixed
+ * 256 KiB device array of the library, which every GPU that loads the library holds
+ * until the process exits.
+ *   - The first call made with a device current looks the array's address up on that
+ *     device; make that first call before any stream capture.
+ *   - Every call rewrites the array (table for its own parameters, error word cleared),
+ *     so calls whose GPU work overlaps (other streams, other threads) race: order them
+ *     on one stream.
+ *   - The array holds RoPE positions 0..510: configurations whose candidate lists can
+ *     exceed 510 entries ((top_k + 1) * branching, bounded by the capacity) return
+ *     RECSA_ERR_UNSUPPORTED with nothing launched.
+ *   - Device-side checks are not reported: the error word is cleared by the next call. */
+RECSA_API recsa_status recsa_decode_no_alloc(const recsa_params *params, const recsa_tree *tree, const void *q,
+                                             int32_t num_queries, void *out, int32_t out_is_fp32,
+                                             recsa_stream_t stream);
+
 /* Synchronise `stream`, then read and clear the workspace's device error word.
  * Returns RECSA_OK, RECSA_ERR_DEVICE_CHECK (an index out of range, or a workspace
  * that was not initialised for the call), RECSA_ERR_TIMEOUT (a bounded wait ran

@@ -29,7 +29,7 @@ def test_library_exports_every_declared_symbol():
     names = declared_functions()
     assert set(names) == {"recsa_tree_layout", "recsa_workspace_size", "recsa_workspace_init", "recsa_build_tree",
                           "recsa_decode", "recsa_prefill_chunk", "recsa_check_device_errors", "recsa_status_string",
-                          "recsa_last_error"}, names
+                          "recsa_last_error", "recsa_decode_no_alloc"}, names
     for n in names:
         assert hasattr(lib, n), n
         assert ctypes.cast(getattr(lib, n), ctypes.c_void_p).value
