@@ -447,12 +447,18 @@ __device__ __forceinline__ void store_out4(const AttendArgs &a, int64_t at, floa
 // ================================================================== CTA / cluster kernel
 
 struct CtaLayout {
-  int misc, geo, q, cand, skey, rank, slog, red, clm, total;
+  int misc, geo, q, cand, skey, rank, slog, ownk, fkey, fpos, kflag, red, clm, fin_cap, total;
 };
+
+// Finalists per level (two-stage selection): every CTA publishes the top k of each group
+// of 32 of its own rows; used while top_k <= 32.
+__host__ __device__ inline int finalist_cap(int CS, int own_max, int top_k) {
+  return (top_k >= 1 && top_k <= 32) ? CS * ((own_max + 31) / 32) * top_k : 0;
+}
 
 __host__ __device__ inline int align128(int x) { return (x + 127) & ~127; }
 
-__host__ __device__ inline CtaLayout cta_layout(int G, int CS, int max_cand, int own_max) {
+__host__ __device__ inline CtaLayout cta_layout(int G, int CS, int max_cand, int own_max, int top_k) {
   CtaLayout L;
   int o = 0;
   auto take = [&o](int bytes) {
@@ -467,6 +473,11 @@ __host__ __device__ inline CtaLayout cta_layout(int G, int CS, int max_cand, int
   L.skey = take((CS > 1 ? 2 : 1) * max_cand * 4);
   L.rank = take(max_cand * 4);
   L.slog = take(2 * G * own_max * 4);  // by level parity: the next level scores while this one folds
+  L.fin_cap = finalist_cap(CS, own_max, top_k);
+  L.ownk = L.fin_cap ? take(own_max * 4) : 0;  // own keys: only the finalist path reads them
+  L.fkey = take(2 * L.fin_cap * 4);  // by level parity: peers publish the next level's while this one reads
+  L.fpos = take(2 * L.fin_cap * 4);
+  L.kflag = take(L.fin_cap * 4 + 4);
   L.red = take(kCtaWarps * G * kRedStride * 4);
   L.clm = CS > 1 ? take(CS * G * kRedStride * 4) : 0;
   L.total = o;
@@ -492,7 +503,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const Attend
   constexpr int PASS = kHalfWarps * RPH;              // rows per CTA per pass
   constexpr bool PIPE = RPH == 2;                      // gather the next level before folding this one
   extern __shared__ __align__(128) unsigned char smem[];
-  const CtaLayout Ls = cta_layout(G, CS, a.max_cand, a.own_max);
+  const CtaLayout Ls = cta_layout(G, CS, a.max_cand, a.own_max, a.top_k);
   int *misc = reinterpret_cast<int *>(smem + Ls.misc);  // [1] ws bad, [2..17] warp totals, [24 + parity] next count
   Geo *geo_s = reinterpret_cast<Geo *>(smem + Ls.geo);
   load_geo(a, geo_s, threadIdx.x, kCtaThreads);
@@ -503,7 +514,11 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const Attend
   uint32_t *skey_all = reinterpret_cast<uint32_t *>(smem + Ls.skey);
   int *rank = reinterpret_cast<int *>(smem + Ls.rank);
   float *slog_all = reinterpret_cast<float *>(smem + Ls.slog);
-  const int OWN = a.own_max, MC = a.max_cand;
+  uint32_t *own_key = reinterpret_cast<uint32_t *>(smem + Ls.ownk);
+  uint32_t *fkey_all = reinterpret_cast<uint32_t *>(smem + Ls.fkey);
+  int *fpos_all = reinterpret_cast<int *>(smem + Ls.fpos);
+  int *kflag = reinterpret_cast<int *>(smem + Ls.kflag);
+  const int OWN = a.own_max, MC = a.max_cand, FCAP = Ls.fin_cap;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int j16 = lane & 15, hw = warp * 2 + (lane >> 4);  // half-warp id 0..15
@@ -628,6 +643,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const Attend
     cand[i] = (uint32_t)i | (i == fpos ? kForced : 0u);
     rank[i] = 0;
   }
+  for (int i = tid; i < 2 * FCAP; i += kCtaThreads) fpos_all[i] = -1;
   if (tid == 0) misc[1] = (hdr_magic != kWsMagic || hdr_rows < a.table_rows_needed) ? 1 : 0;
   __syncthreads();
   if constexpr (CS > 1) cluster_barrier();  // every peer runs before the first DSMEM store
@@ -639,6 +655,14 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const Attend
     float *slog = slog_all + (lvl & 1) * G * OWN;
     const bool single = hi_r - lo_r <= PASS;
     const LevelRows lr = level_rows(a, geo, lvl, t.bh);
+
+    const int nforced = (a.causal && n > 0 && (cl[n - 1] & kForced)) ? 1 : 0;
+    const int m = n - nforced;
+    // two-stage selection: each CTA ranks its own rows within groups of 32 and publishes
+    // the top k of each group as finalists; then every CTA ranks the finalists
+    const int groups = (per + 31) / 32;  // groups per CTA (the same in every CTA)
+    const int nfin = CS * groups * a.top_k;
+    const bool fast = lvl > 0 && single && a.top_k >= 1 && a.top_k < m && nfin <= FCAP && nfin <= kCtaThreads;
 
     // 1. score this CTA's slice (rows preloaded, or gathered now)
     const Trig4 tq = preloaded ? tq_pre : ldg_trig4(a.table, n, j16);
@@ -658,7 +682,10 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const Attend
         if (rs.ok[r]) dot_row8<G>(rs.k[r], rs.tr[r], q2lo, q2hi, part);
         const float x = reduce16<G>(part, j16) * a.scale;
         const float S = group_sum16<G>(x);
-        if (rs.ok[r]) {
+        if (fast) {
+          if (j16 == 0 && rs.pos[r] < hi_r) own_key[rs.pos[r] - lo_r] = rs.ok[r] ? order_key(S) : 0u;
+          if (rs.ok[r] && head_writer<G>(j16)) slog[head_of<G>(j16) * OWN + rs.pos[r] - lo_r] = x;
+        } else if (rs.ok[r]) {
           if (head_writer<G>(j16)) slog[head_of<G>(j16) * OWN + rs.pos[r] - lo_r] = x;
           if (lvl > 0 && j16 == 0) {
             const uint32_t key = order_key(S);
@@ -686,14 +713,104 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const Attend
     // the next count slot of this level's parity was last read two levels ago
     int *next_count = misc + 24 + (lvl & 1);
     if (tid == 0) *next_count = 0;
-    const int nforced = (a.causal && n > 0 && (cl[n - 1] & kForced)) ? 1 : 0;
-    const int m = n - nforced;
     keys_read += m;
+    uint32_t *fkey = fkey_all + (lvl & 1) * FCAP;
+    int *fpos = fpos_all + (lvl & 1) * FCAP;
+    {  // the next level's finalist slots (read last two levels ago) start empty
+      int *fnext = fpos_all + ((lvl - 1) & 1) * FCAP;
+      for (int i = tid; i < FCAP; i += kCtaThreads) fnext[i] = -1;
+    }
+    if (fast) {
+      __syncthreads();  // own keys
+      const int own = hi_r - lo_r;
+      const int tpi = min(32, 1 << (31 - __clz(kCtaThreads / max(own, 1))));  // lanes per item
+      const int item = tid / tpi, q = tid - item * tpi;
+      const uint32_t kc = item < own ? own_key[item] : 0u;
+      const int g0 = item & ~31, gcnt = min(32, own - g0);
+      int better = 0;
+      if (item < own)
+        for (int j = q; j < gcnt; j += tpi) {
+          const uint32_t kj = own_key[g0 + j];
+          better += (kj > kc || (kj == kc && g0 + j < item)) ? 1 : 0;
+        }
+      for (int o = 1; o < tpi; o <<= 1) better += __shfl_xor_sync(0xffffffffu, better, o);
+      if (q == 0 && item < own && kc != 0u && better < a.top_k) {
+        const int slot = (crank * groups + (item >> 5)) * a.top_k + better;
+        if constexpr (CS > 1) {
+          cg::cluster_group cluster = cg::this_cluster();
+#pragma unroll
+          for (int r = 0; r < CS; ++r) {
+            cluster.map_shared_rank(fkey, r)[slot] = kc;
+            cluster.map_shared_rank(fpos, r)[slot] = lo_r + item;
+          }
+        } else {
+          fkey[slot] = kc;
+          fpos[slot] = lo_r + item;
+        }
+      }
+    }
     if constexpr (CS > 1) cluster_barrier();
     __syncthreads();
 
     int n_next = 0;
-    if (lvl > 0) {
+    if (fast) {
+      // 2'. rank the finalists; the kept ones, in node order, expand into the next list
+      const int tpi = min(32, 1 << (31 - __clz(kCtaThreads / nfin)));
+      const int f = tid / tpi, q = tid - f * tpi;
+      const int pf = f < nfin ? fpos[f] : -1;
+      const uint32_t kf = f < nfin ? fkey[f] : 0u;
+      int better = 0;
+      if (pf >= 0)
+        for (int j = q; j < nfin; j += tpi) {
+          const int pj = fpos[j];
+          const uint32_t kj = fkey[j];
+          better += (pj >= 0 && (kj > kf || (kj == kf && pj < pf))) ? 1 : 0;
+        }
+      for (int o = 1; o < tpi; o <<= 1) better += __shfl_xor_sync(0xffffffffu, better, o);
+      const bool kept = pf >= 0 && better < a.top_k;
+      if (q == 0 && f < nfin) kflag[f] = kept ? 1 : 0;
+      const int nkept = __syncthreads_count(q == 0 && kept);
+      int32_t *sel = (a.sel_idx != nullptr && crank == 0 && lvl <= a.sel_levels)
+                         ? a.sel_idx + ((int64_t)tile * a.sel_levels + (lvl - 1)) * a.top_k
+                         : nullptr;
+      if (sel)
+        for (int u = nkept + tid; u < a.top_k; u += kCtaThreads) sel[u] = -1;
+      uint32_t *nx = cand + (cur ^ 1) * MC;
+      const LevelRows lb = level_rows(a, geo, lvl - 1, t.bh);
+      auto expand_one = [&](uint32_t v, int e) {  // children of the e-th expanded node
+        bool lf = false;
+        const int nch = child_count(a, geo, v, lvl, t.p, &lf);
+        const int off = e * a.b;
+        const int first = (int)(v & kNodeMask) * a.b;
+        for (int u = 0; u < nch && off + u < MC; ++u)
+          nx[off + u] = (uint32_t)(first + u) | ((lf && u == nch - 1) ? kForced : 0u);
+        if (off + nch > MC) atomicOr(err, kErrCount);
+        atomicMax(next_count, min(off + nch, MC));
+        if (nch > 0 && e % CS == crank && first + nch <= lb.nrows) {
+          prefetch_l2(lb.k + (int64_t)first * kD, (uint32_t)nch * kRowBytes);
+          prefetch_l2(lb.v + (int64_t)first * kD, (uint32_t)nch * kRowBytes);
+        }
+      };
+      int e = 0;
+      if (kept)
+        for (int j = q; j < nfin; j += tpi) e += (kflag[j] && fpos[j] < pf) ? 1 : 0;
+      for (int o = 1; o < tpi; o <<= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+      if (kept && q == 0) {
+        const uint32_t v = cl[pf];
+        cl[pf] = v | kKept;
+        if (sel) sel[e] = (int32_t)(v & kNodeMask);
+        expand_one(v, e);
+      }
+      if (nforced && tid == kCtaThreads - 1) expand_one(cl[n - 1], nkept);
+      values_read += m - a.top_k;
+      __syncthreads();
+      n_next = min(*next_count, MC);
+      if (n_next > a.table_rows_needed - 1) {
+        if (tid == 0) atomicOr(err, kErrCount);
+        n_next = a.table_rows_needed - 1;
+      }
+      for (int i = tid; i < n_next; i += kCtaThreads) rank[i] = 0;
+    } else if (lvl > 0) {
       // 2. top-k by rank: a candidate is kept when fewer than k scorable candidates beat it
       const bool keep_all = a.top_k >= m;
       if (!keep_all && a.top_k > 0) {
@@ -839,6 +956,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const Attend
       }
     }
     n = n_next;
+    per = per2;
     lo_r = lo2;
     hi_r = hi2;
     cur ^= 1;
@@ -1159,7 +1277,7 @@ template <int G, int CS>
 int launch_cta(const AttendArgs &args, cudaStream_t stream) {
   AttendArgs a = args;
   a.own_max = ((a.max_cand + CS - 1) / CS + 31) / 32 * 32;
-  const CtaLayout L = cta_layout(G, CS, a.max_cand, a.own_max);
+  const CtaLayout L = cta_layout(G, CS, a.max_cand, a.own_max, a.top_k);
   if (L.total > 227 * 1024) {
     set_error("attend needs %d bytes of shared memory per CTA (limit 232448)", L.total);
     return -1;
