@@ -137,12 +137,20 @@ class Timer:
 
 
 def max_over_ranks(x: float, dist_on: bool) -> float:
+    """Largest value over all ranks (every rank gets it); identity on one process."""
     if not dist_on:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank_step: int, steps: int, local_seconds: float, world: int, dist_on: bool):
+    """Whole-job units/s of independent replicas: all ranks' units over the slowest rank's time."""
+    slowest = max_over_ranks(local_seconds, dist_on)
+    return world * units_per_rank_step * steps / slowest, slowest
 
 
 def pct(xs, q):
@@ -483,7 +491,7 @@ def run_gpu(args):
         return
     B = w.batch
     n = world
-    value = n * dec["queries"] * args.steps / dec["total_s"]
+    value = n * dec["queries"] * args.steps / dec["total_s"]  # total_s is already the max over ranks
     mean_s = dec["mean_s"]
     achieved = dec["bytes_per_launch"] / mean_s / 1e9
     traffic = recorded_traffic("decode_1m_attend_traffic")

@@ -49,6 +49,10 @@ constexpr int kWarpKernelMaxWarps = 8;
 constexpr int kTopkRegs = 8;                        // iterative top-k handles up to 256 candidates
 // merge rows: m, l, 2 pad, acc[128] (the accumulator starts 16-byte aligned)
 constexpr int kRedStride = kD + 4;
+// CTA kernel scratch ints: [1] workspace bad, [2, 2 + 2W) per-warp ballot totals,
+// [kNextCount + parity] next level's candidate count
+constexpr int kNextCount = 2 + 2 * (kCtaThreads / 32);
+constexpr int kMiscInts = kNextCount + 2;
 
 struct AttendArgs {
   const uint16_t *k_tok, *v_tok, *k_node, *v_node;
@@ -184,7 +188,7 @@ __device__ __forceinline__ Row8 ldg_row8(const uint16_t *row, int j16) {
 }
 
 struct Trig4 {
-  float4 a, b;  // (cos, sin) of the 4 frequencies 4j..4j+3
+  float4 a, b;  // frequencies (4j, 4j+1) and (4j+2, 4j+3): (cos, cos', sin, sin') each
 };
 
 __device__ __forceinline__ Trig4 ldg_trig4(const float2 *table, int pos, int j16) {
@@ -208,8 +212,8 @@ __device__ __forceinline__ void unpack_row8(const Row8 &r, float (&lo)[4], float
 
 // rotate-half RoPE of the 4 pairs (lo[t], hi[t]): lo' = lo c - hi s, hi' = hi c + lo s
 __device__ __forceinline__ void rotate4(float (&lo)[4], float (&hi)[4], const Trig4 &tr) {
-  const float c[4] = {tr.a.x, tr.a.z, tr.b.x, tr.b.z};
-  const float s[4] = {tr.a.y, tr.a.w, tr.b.y, tr.b.w};
+  const float c[4] = {tr.a.x, tr.a.y, tr.b.x, tr.b.y};
+  const float s[4] = {tr.a.z, tr.a.w, tr.b.z, tr.b.w};
 #pragma unroll
   for (int t = 0; t < 4; ++t) {
     const float l = lo[t], h = hi[t];
@@ -466,7 +470,7 @@ __host__ __device__ inline CtaLayout cta_layout(int G, int CS, int max_cand, int
     o = align128(o + bytes);
     return r;
   };
-  L.misc = take(128);
+  L.misc = take(kMiscInts * 4);
   L.geo = take(kGeoBytes);
   L.q = take(G * kD * 4);
   L.cand = take(2 * max_cand * 4);
@@ -504,7 +508,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const Attend
   constexpr bool PIPE = RPH == 2;                      // gather the next level before folding this one
   extern __shared__ __align__(128) unsigned char smem[];
   const CtaLayout Ls = cta_layout(G, CS, a.max_cand, a.own_max, a.top_k);
-  int *misc = reinterpret_cast<int *>(smem + Ls.misc);  // [1] ws bad, [2..17] warp totals, [24 + parity] next count
+  int *misc = reinterpret_cast<int *>(smem + Ls.misc);  // see kMiscInts
   Geo *geo_s = reinterpret_cast<Geo *>(smem + Ls.geo);
   load_geo(a, geo_s, threadIdx.x, kCtaThreads);
   __syncthreads();
@@ -711,7 +715,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const Attend
     }
     preloaded = false;
     // the next count slot of this level's parity was last read two levels ago
-    int *next_count = misc + 24 + (lvl & 1);
+    int *next_count = misc + kNextCount + (lvl & 1);
     if (tid == 0) *next_count = 0;
     keys_read += m;
     uint32_t *fkey = fkey_all + (lvl & 1) * FCAP;
@@ -749,8 +753,11 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const Attend
         }
       }
     }
-    if constexpr (CS > 1) cluster_barrier();
-    __syncthreads();
+    if constexpr (CS > 1) {
+      cluster_barrier();  // also orders this CTA's shared memory (release/acquire)
+    } else {
+      __syncthreads();
+    }
 
     int n_next = 0;
     if (fast) {

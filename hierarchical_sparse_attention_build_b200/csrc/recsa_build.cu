@@ -157,15 +157,20 @@ __global__ void append_kernel(const uint4 *__restrict__ k_new, const uint4 *__re
   }
 }
 
-// RoPE table: table[pos][i] = (cos, sin)(pos * base^(-2i/128)), computed in fp64.
-__global__ void rope_table_kernel(float2 *table, int rows, double base, WsHeader *hdr) {
+// RoPE table, computed in fp64 and stored fp32: for position pos and frequency pair u
+// (frequencies 2u, 2u+1, angle pos * base^(-2i/128)) the four floats
+// table[pos][u] = (cos_2u, cos_2u+1, sin_2u, sin_2u+1), so a pair of frequencies loads
+// as packed (cos, cos') and (sin, sin') operands.
+__global__ void rope_table_kernel(float *table, int rows, double base, WsHeader *hdr) {
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx < rows * kHalf) {
     const int pos = idx / kHalf, i = idx % kHalf;
     const double inv_freq = pow(base, -2.0 * (double)i / (double)kD);
     double s, c;
     sincos((double)pos * inv_freq, &s, &c);
-    table[idx] = make_float2((float)c, (float)s);
+    float *pair = table + (size_t)pos * (2 * kHalf) + (i >> 1) * 4 + (i & 1);
+    pair[0] = (float)c;
+    pair[2] = (float)s;
   }
   if (idx == 0) {
     hdr->err = 0u;
@@ -187,7 +192,7 @@ int sm_count() {
 
 int launch_rope_table(void *ws, int rows, double base, void *stream) {
   auto *hdr = reinterpret_cast<WsHeader *>(ws);
-  auto *table = reinterpret_cast<float2 *>(reinterpret_cast<char *>(ws) + kWsHeader);
+  auto *table = reinterpret_cast<float *>(reinterpret_cast<char *>(ws) + kWsHeader);
   const int n = rows * kHalf;
   const int threads = 256;
   const int blocks = (n + threads - 1) / threads;
