@@ -515,7 +515,7 @@ def run_gpu(args):
                    "l2": "flushed between timed steps (256 MiB write, untimed)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": traffic,
-                     "kernel": "attend_cta_kernel<4,4> (recsa_decode, 4-CTA clusters)",
+                     "kernel": "attend_lean_kernel<4,4,2> (recsa_decode, 4-CTA clusters)",
                      "algorithmic_bytes_per_launch": dec["bytes_per_launch"],
                      "peak_source": f"{peaks_src} hbm_gbs (MEASURED_PEAKS.json)"},
         "e2e": {"value": n * dec["queries"] * args.steps / dec["e2e_total_s"], "unit": "queries/s",

@@ -76,7 +76,7 @@ class Debug(ctypes.Structure):
     ]
 
 
-KERNEL_AUTO, KERNEL_CTA, KERNEL_WARP = 0, 1, 2
+KERNEL_AUTO, KERNEL_CTA, KERNEL_WARP, KERNEL_LEAN = 0, 1, 2, 3
 
 
 def _load() -> ctypes.CDLL:

@@ -44,7 +44,6 @@ constexpr uint32_t kNodeMask = 0x3fffffffu;
 constexpr int kCtaThreads = 256;
 constexpr int kCtaWarps = kCtaThreads / 32;
 constexpr int kHalfWarps = 2 * kCtaWarps;           // 16 row slots per CTA
-constexpr int kPassRows = 2 * kHalfWarps;           // rows a CTA holds per pass (2 per half-warp)
 constexpr int kWarpKernelMaxWarps = 8;
 constexpr int kTopkRegs = 8;                        // iterative top-k handles up to 256 candidates
 // merge rows: m, l, 2 pad, acc[128] (the accumulator starts 16-byte aligned)
@@ -1054,6 +1053,469 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const Attend
   if (ws_bad && tid == 0 && crank == 0) atomicOr(err, kErrWs);
 }
 
+// ================================================================== lean cluster kernel
+//
+// One cluster of CS CTAs per tile, one memory round trip, one cluster barrier and one
+// block barrier per level.  Every CTA holds the rows of its slice of the level in
+// registers; it scores them and stores each group score into every CTA of the cluster;
+// after the cluster barrier each CTA ranks all n scores itself, so every CTA knows the
+// kept set without a second exchange.  The next level's rows are addressed
+// straight from the kept mask (child i of the level belongs to the (i / b)-th expanded
+// node), issued, and only then is this level's unkept part folded.
+
+constexpr int kLeanMaxCand = 256;  // candidates per level the lean kernel ranks (one bit each)
+
+struct LeanLayout {
+  int geo, kbuf, mask, par, red, clm, total;
+};
+
+__host__ __device__ inline LeanLayout lean_layout(int G, int CS, int max_cand) {
+  LeanLayout L;
+  int o = 0;
+  auto take = [&o](int bytes) {
+    const int r = o;
+    o = align128(o + bytes);
+    return r;
+  };
+  L.geo = take(kGeoBytes);
+  L.kbuf = take(2 * kLeanMaxCand * 4);  // group scores (order keys) by level parity
+  L.mask = take(2 * 16 * 2);            // kept bits, 16 per half-word, by level parity
+  L.par = take(2 * max_cand * 4);       // expanded node ids of the level above, by parity
+  L.red = take(kCtaWarps * G * kRedStride * 4);
+  L.clm = take(CS * G * kRedStride * 4);
+  L.total = o;
+  return L;
+}
+
+// #{j in [j0, j1) : k[j] > thr}
+__device__ __forceinline__ int count_above(const uint32_t *k, int j0, int j1, uint32_t thr) {
+  int cnt = 0, j = j0;
+  for (; j < j1 && (j & 3); ++j) cnt += k[j] > thr;
+  for (; j + 4 <= j1; j += 4) {
+    const uint4 v = *reinterpret_cast<const uint4 *>(k + j);
+    cnt += (v.x > thr) + (v.y > thr) + (v.z > thr) + (v.w > thr);
+  }
+  for (; j < j1; ++j) cnt += k[j] > thr;
+  return cnt;
+}
+
+// Position of the e-th (0-based) set bit of the 256-bit mask w; e < popcount(w).
+__device__ __forceinline__ int nth_set(const uint32_t (&w)[8], int e) {
+  int base = 0;
+  uint32_t x = 0;
+  bool found = false;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int c = __popc(w[i]);
+    if (!found) {
+      if (e < c) {
+        x = w[i];
+        base = i * 32;
+        found = true;
+      } else {
+        e -= c;
+      }
+    }
+  }
+  int pos = 0;
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) {
+    const int c = __popc(x & ((1u << s) - 1u));
+    if (e >= c) {
+      e -= c;
+      x >>= s;
+      pos += s;
+    }
+  }
+  return base + pos;
+}
+
+__device__ __forceinline__ bool bit_of(const uint32_t (&w)[8], int pos) {
+  uint32_t x = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) x = (i == (pos >> 5)) ? w[i] : x;
+  return (x >> (pos & 31)) & 1u;
+}
+
+template <int G>
+__device__ __forceinline__ void rotated_query_regs(const uint2 (&qlo)[G], const uint2 (&qhi)[G], const Trig4 &tq,
+                                                   float2 (&q2lo)[G][2], float2 (&q2hi)[G][2]) {
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    float lo[4], hi[4];
+    Row8 r;
+    r.lo = qlo[h];
+    r.hi = qhi[h];
+    unpack_row8(r, lo, hi);
+    rotate4(lo, hi, tq);
+    q2lo[h][0] = make_float2(lo[0], lo[1]);
+    q2lo[h][1] = make_float2(lo[2], lo[3]);
+    q2hi[h][0] = make_float2(hi[0], hi[1]);
+    q2hi[h][1] = make_float2(hi[2], hi[3]);
+  }
+}
+
+// Every slice of a level fits in RPH rows per half-warp: ceil(max_cand / CS) <= 16 RPH,
+// and max_cand <= kLeanMaxCand (the launcher checks both).
+template <int G, int CS, int RPH>
+__global__ void __launch_bounds__(kCtaThreads, 1) attend_lean_kernel(const AttendArgs a) {
+  static_assert(CS == 2 || CS == 4, "the lean kernel runs in clusters of 2 or 4");
+  constexpr unsigned F = 0xffffffffu;
+  extern __shared__ __align__(128) unsigned char smem[];
+  const LeanLayout Ls = lean_layout(G, CS, a.max_cand);
+  Geo *geo_s = reinterpret_cast<Geo *>(smem + Ls.geo);
+  uint32_t *kbuf = reinterpret_cast<uint32_t *>(smem + Ls.kbuf);
+  uint16_t *mask16 = reinterpret_cast<uint16_t *>(smem + Ls.mask);
+  int *par_all = reinterpret_cast<int *>(smem + Ls.par);
+  float *red = reinterpret_cast<float *>(smem + Ls.red);  // [warp][h][kRedStride]: m, l, pad, acc[128]
+  float *clm = reinterpret_cast<float *>(smem + Ls.clm);  // [rank][h][kRedStride], read on rank 0
+  const int MC = a.max_cand;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int j16 = lane & 15, hw = warp * 2 + (lane >> 4);
+  const int crank = (int)cg::this_cluster().block_rank();
+  const int tile = blockIdx.x / CS;
+  uint32_t *err = &a.hdr->err;
+
+  cg::cluster_group cluster = cg::this_cluster();
+  load_geo(a, geo_s, tid, kCtaThreads);
+  __syncthreads();
+  const Geo &geo = *geo_s;
+  const TileInfo t = tile_info(a, geo, tile);
+  const int64_t out0 = (((int64_t)t.s * a.nq + t.qi) * a.hq + (int64_t)t.g * G) * kD;
+  // lane j16 < CS stores the scores of its half-warp's rows into cluster CTA j16
+  uint32_t *dst_kbuf = cluster.map_shared_rank(kbuf, (unsigned)(j16 % CS));
+  // floor(x / b) = umulhi(x, bmagic) for 0 <= x < 2^32 / b
+  const uint32_t bmagic = 0xffffffffu / (uint32_t)a.b + 1u;
+  auto divb = [&](int x) { return (int)__umulhi((uint32_t)x, bmagic); };
+
+  // the query heads of the group: dims 4j..4j+3 and 64+4j..64+4j+3 (bf16 pairs)
+  uint2 qlo[G], qhi[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    qlo[h] = __ldg(reinterpret_cast<const uint2 *>(a.q + out0 + h * kD + 4 * j16));
+    qhi[h] = __ldg(reinterpret_cast<const uint2 *>(a.q + out0 + h * kD + kHalf + 4 * j16));
+  }
+
+  int fpos;
+  int n = top_candidates(a, geo, t, &fpos);
+  const int n_cap = min(MC, a.table_rows_needed - 1);
+  if (n > n_cap) {  // cannot happen for a valid launch; guards the buffers and the table
+    if (tid == 0) atomicOr(err, kErrCount);
+    n = n_cap;
+  }
+  if (fpos >= n) fpos = -1;
+
+  Row8 ck[RPH], cv[RPH], nk[RPH], nv[RPH];
+  Trig4 ctr[RPH], ntr[RPH];
+  bool cok[RPH], nok[RPH];
+  auto load_row = [&](const LevelRows &lr, int pos, int node, bool valid, Row8 &k, Row8 &v, Trig4 &tr, bool &ok) {
+    ok = valid && node >= 0 && node < lr.nrows;
+    if (valid && !ok && j16 == 0) atomicOr(err, kErrIndex);
+    if (ok) {
+      k = ldg_row8(lr.k + (int64_t)node * kD, j16);
+      v = ldg_row8(lr.v + (int64_t)node * kD, j16);
+      tr = ldg_trig4(a.table, pos, j16);
+    }
+  };
+  // node of candidate `pos` of the current level: the top level lists its nodes in
+  // order; below, candidate i is child i % b of the (i / b)-th expanded node above
+  auto cand_node = [&](const int *par, bool top, int pos) -> int {
+    if (top) return pos;
+    const int e = divb(pos);
+    return par[e] * a.b + (pos - e * a.b);
+  };
+
+  int per = (n + CS - 1) / CS;
+  int lo = min(n, crank * per), hi = min(n, lo + per);
+  {
+    const LevelRows lr = level_rows(a, geo, t.T, t.bh);
+#pragma unroll
+    for (int r = 0; r < RPH; ++r) {
+      const int pos = lo + hw + kHalfWarps * r;
+      load_row(lr, pos, pos, pos < hi && pos != fpos, ck[r], cv[r], ctr[r], cok[r]);
+    }
+  }
+  Trig4 tq = ldg_trig4(a.table, n, j16), ntq;
+  cluster_barrier();  // every CTA of the cluster runs before the first store into a peer
+
+  float m_w[G], l_w[G];
+  float2 acc[G][4];  // dims (4j, 4j+1), (4j+2, 4j+3), (64+4j, ..), (64+4j+2, ..)
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    m_w[h] = -INFINITY;
+    l_w[h] = 0.f;
+#pragma unroll
+    for (int d = 0; d < 4; ++d) acc[h][d] = make_float2(0.f, 0.f);
+  }
+  int keys_read = 0, values_read = 0;
+
+  // Fold the entry rows (values in registers, logits of every head in xs) into the
+  // half-warp's online-softmax state.
+  auto fold = [&](const Row8 (&vr)[RPH], const float (&xs)[RPH][G], const bool (&ent)[RPH]) {
+    float mnew[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float mx = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < RPH; ++r)
+        if (ent[r]) mx = fmaxf(mx, xs[r][h]);
+      mx = fmaxf(mx, __shfl_xor_sync(F, mx, 16));
+      mnew[h] = fmaxf(m_w[h], mx);
+      const float alpha = (mnew[h] == -INFINITY) ? 1.f : __expf(m_w[h] - mnew[h]);
+      m_w[h] = mnew[h];
+      l_w[h] *= alpha;
+      const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+      for (int d = 0; d < 4; ++d) acc[h][d] = __fmul2_rn(acc[h][d], a2);
+    }
+    float ls[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) ls[h] = 0.f;
+#pragma unroll
+    for (int r = 0; r < RPH; ++r)
+      if (ent[r]) {
+        const Row8 &v = vr[r];
+        const float2 v0 = make_float2(bf16_lo(v.lo.x), bf16_hi(v.lo.x)), v1 = make_float2(bf16_lo(v.lo.y), bf16_hi(v.lo.y));
+        const float2 v2 = make_float2(bf16_lo(v.hi.x), bf16_hi(v.hi.x)), v3 = make_float2(bf16_lo(v.hi.y), bf16_hi(v.hi.y));
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float pr = __expf(xs[r][h] - mnew[h]);
+          ls[h] += pr;
+          const float2 p2 = make_float2(pr, pr);
+          acc[h][0] = __ffma2_rn(p2, v0, acc[h][0]);
+          acc[h][1] = __ffma2_rn(p2, v1, acc[h][1]);
+          acc[h][2] = __ffma2_rn(p2, v2, acc[h][2]);
+          acc[h][3] = __ffma2_rn(p2, v3, acc[h][3]);
+        }
+      }
+#pragma unroll
+    for (int h = 0; h < G; ++h) l_w[h] += ls[h] + __shfl_xor_sync(F, ls[h], 16);
+  };
+
+  for (int j = 0, lvl = t.T;; ++j, --lvl) {
+    const int pb = j & 1;
+    const bool top = lvl == t.T;
+    const int *par_cur = par_all + pb * MC;  // written one level up (unused at the top)
+    // 1. scores of this CTA's rows: logits of every head (xs) and the group score key
+    float xs[RPH][G];
+    uint32_t key[RPH];
+    {
+      float2 q2lo[G][2], q2hi[G][2];
+      rotated_query_regs<G>(qlo, qhi, tq, q2lo, q2hi);
+#pragma unroll
+      for (int r = 0; r < RPH; ++r) {
+        float part[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) part[h] = 0.f;
+        if (cok[r]) dot_row8<G>(ck[r], ctr[r], q2lo, q2hi, part);
+        const float x = reduce16<G>(part, j16) * a.scale;
+        const float S = group_sum16<G>(x);  // shuffles: every lane, row or not
+        key[r] = cok[r] ? order_key(S) : 0u;
+#pragma unroll
+        for (int h = 0; h < G; ++h) xs[r][h] = __shfl_sync(F, x, (lane & 16) | (h << (4 - log2g<G>())));
+      }
+    }
+    const int m = n - (fpos >= 0 ? 1 : 0);
+    keys_read += m;
+    bool ent[RPH];
+    if (lvl == 0) {
+      values_read += n;
+#pragma unroll
+      for (int r = 0; r < RPH; ++r) ent[r] = cok[r];
+      fold(cv, xs, ent);
+      break;
+    }
+
+    // 2. the group scores go to every CTA of the cluster (lane j16 < CS of each
+    //    half-warp into CTA j16); the barrier publishes them
+    if (j16 < CS) {
+#pragma unroll
+      for (int r = 0; r < RPH; ++r) {
+        const int pos = lo + hw + kHalfWarps * r;
+        if (pos < hi) dst_kbuf[pb * kLeanMaxCand + pos] = key[r];
+      }
+    }
+    cluster_barrier();
+
+    // 3. rank: candidate c is kept when fewer than top_k scorable candidates beat it
+    //    (higher score, or equal score at a lower position)
+    {
+      const uint32_t *kb = kbuf + pb * kLeanMaxCand;
+      int c, j0, j1;
+      if (n <= 128) {  // two threads per candidate, half the competitors each
+        c = warp * 16 + j16;
+        const int h2 = (((n + 1) >> 1) + 3) & ~3;
+        j0 = min(n, (lane >> 4) * h2);
+        j1 = min(n, j0 + h2);
+      } else {
+        c = tid;
+        j0 = 0;
+        j1 = n;
+      }
+      const uint32_t kc = c < n ? kb[c] : 0u;
+      int better = count_above(kb, j0, min(j1, max(j0, c)), kc - 1u) + count_above(kb, max(j0, min(j1, c + 1)), j1, kc);
+      if (n <= 128) better += __shfl_xor_sync(F, better, 16);
+      const unsigned bal = __ballot_sync(F, c < n && kc != 0u && better < a.top_k);
+      if (lane == 0) {
+        uint16_t *mk = mask16 + pb * 16;
+        if (n <= 128) {
+          mk[warp] = (uint16_t)(bal & 0xffffu);
+        } else {
+          mk[2 * warp] = (uint16_t)(bal & 0xffffu);
+          mk[2 * warp + 1] = (uint16_t)(bal >> 16);
+        }
+      }
+    }
+    __syncthreads();
+    uint32_t kw[8], ew[8];
+    {
+      const uint4 w0 = *reinterpret_cast<const uint4 *>(mask16 + pb * 16);
+      uint4 w1 = make_uint4(0u, 0u, 0u, 0u);
+      if (n > 128) w1 = *reinterpret_cast<const uint4 *>(mask16 + pb * 16 + 8);
+      kw[0] = w0.x, kw[1] = w0.y, kw[2] = w0.z, kw[3] = w0.w;
+      kw[4] = w1.x, kw[5] = w1.y, kw[6] = w1.z, kw[7] = w1.w;
+    }
+    int nK = 0, nE = 0, last = -1;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      ew[i] = kw[i] | ((fpos >= 0 && (fpos >> 5) == i) ? (1u << (fpos & 31)) : 0u);
+      nK += __popc(kw[i]);
+      nE += __popc(ew[i]);
+      if (ew[i]) last = i * 32 + 31 - __clz(ew[i]);
+    }
+    values_read += m - min(a.top_k, m);
+
+    // 4. the next level: its size, forced node, this CTA's slice, and the slice's rows
+    int n_next = 0, fpos_next = -1;
+    if (last >= 0) {
+      bool lf = false;
+      const int nch =
+          child_count(a, geo, (uint32_t)cand_node(par_cur, top, last) | (last == fpos ? kForced : 0u), lvl, t.p, &lf);
+      n_next = (nE - 1) * a.b + nch;
+      if (lf) fpos_next = n_next - 1;
+    }
+    if (n_next > n_cap) {
+      if (tid == 0) atomicOr(err, kErrCount);
+      n_next = n_cap;
+      if (fpos_next >= n_next) fpos_next = -1;
+    }
+    const int per2 = (n_next + CS - 1) / CS;
+    const int lo2 = min(n_next, crank * per2), hi2 = min(n_next, lo2 + per2);
+    {
+      const LevelRows lb = level_rows(a, geo, lvl - 1, t.bh);
+#pragma unroll
+      for (int r = 0; r < RPH; ++r) {
+        const int i = lo2 + hw + kHalfWarps * r;
+        const bool valid = i < hi2 && i != fpos_next;
+        int node = 0;
+        if (valid) {
+          const int e = divb(i);
+          node = cand_node(par_cur, top, nth_set(ew, e)) * a.b + (i - e * a.b);
+        }
+        load_row(lb, i, node, valid, nk[r], nv[r], ntr[r], nok[r]);
+      }
+      ntq = ldg_trig4(a.table, n_next, j16);
+    }
+    if (tid < nE) par_all[(pb ^ 1) * MC + tid] = cand_node(par_cur, top, nth_set(ew, tid));
+    if (a.sel_idx != nullptr && crank == 0 && lvl <= a.sel_levels) {
+      int32_t *sel = a.sel_idx + ((int64_t)tile * a.sel_levels + (lvl - 1)) * a.top_k;
+      for (int u = tid; u < a.top_k; u += kCtaThreads) sel[u] = u < nK ? cand_node(par_cur, top, nth_set(kw, u)) : -1;
+    }
+
+    // 5. fold this level's unkept candidates while the next level's rows are in flight
+#pragma unroll
+    for (int r = 0; r < RPH; ++r) ent[r] = cok[r] && !bit_of(kw, lo + hw + kHalfWarps * r);
+    fold(cv, xs, ent);
+
+#pragma unroll
+    for (int r = 0; r < RPH; ++r) {
+      ck[r] = nk[r];
+      cv[r] = nv[r];
+      ctr[r] = ntr[r];
+      cok[r] = nok[r];
+    }
+    tq = ntq;
+    n = n_next;
+    fpos = fpos_next;
+    lo = lo2;
+    hi = hi2;
+  }
+
+  if (a.entries != nullptr && crank == 0 && tid == 0) {
+    a.entries[2 * (int64_t)tile] = keys_read;
+    a.entries[2 * (int64_t)tile + 1] = values_read;
+  }
+
+  // merge: half-warps -> warp -> CTA (here) -> cluster (on rank 0)
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    float2 x[4];
+#pragma unroll
+    for (int d = 0; d < 4; ++d) {
+      x[d].x = acc[h][d].x + __shfl_xor_sync(F, acc[h][d].x, 16);
+      x[d].y = acc[h][d].y + __shfl_xor_sync(F, acc[h][d].y, 16);
+    }
+    float *r = red + (warp * G + h) * kRedStride;
+    if (lane == 0) {
+      r[0] = m_w[h];
+      r[1] = l_w[h];
+    }
+    if (lane < 16) {
+      *reinterpret_cast<float4 *>(r + 4 + 4 * j16) = make_float4(x[0].x, x[0].y, x[1].x, x[1].y);
+      *reinterpret_cast<float4 *>(r + 4 + kHalf + 4 * j16) = make_float4(x[2].x, x[2].y, x[3].x, x[3].y);
+    }
+  }
+  __syncthreads();
+  float *dst_clm = cluster.map_shared_rank(clm, 0u);
+  for (int e = tid; e < G * kD / 4; e += kCtaThreads) {
+    const int h = (4 * e) / kD, d0 = (4 * e) % kD;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kCtaWarps; ++w) M = fmaxf(M, red[(w * G + h) * kRedStride]);
+    float l = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kCtaWarps; ++w) {
+        const float *r = red + (w * G + h) * kRedStride;
+        const float f = (r[0] == -INFINITY) ? 0.f : __expf(r[0] - M);
+        l += f * r[1];
+#pragma unroll
+        for (int d = 0; d < 4; ++d) o[d] += f * r[4 + d0 + d];
+      }
+    }
+    float *dst = dst_clm + (crank * G + h) * kRedStride;
+    if (d0 == 0) {
+      dst[0] = M;
+      dst[1] = l;
+    }
+    *reinterpret_cast<float4 *>(dst + 4 + d0) = make_float4(o[0], o[1], o[2], o[3]);
+  }
+  cluster_barrier();  // every partial is in rank 0; no CTA stores into a peer after this
+  if (crank == 0) {
+    const bool ws_bad = !workspace_ok(a);
+    for (int e = tid; e < G * kD / 4; e += kCtaThreads) {
+      const int h = (4 * e) / kD, d0 = (4 * e) % kD;
+      float M = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < CS; ++r) M = fmaxf(M, clm[(r * G + h) * kRedStride]);
+      float l = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int r = 0; r < CS; ++r) {
+          const float *x = clm + (r * G + h) * kRedStride;
+          const float f = (x[0] == -INFINITY) ? 0.f : __expf(x[0] - M);
+          l += f * x[1];
+#pragma unroll
+          for (int d = 0; d < 4; ++d) o[d] += f * x[4 + d0 + d];
+        }
+      }
+      const float inv = (l > 0.f && !ws_bad) ? 1.f / l : 0.f;
+      store_out4(a, out0 + 4 * e, o[0] * inv, o[1] * inv, o[2] * inv, o[3] * inv);
+    }
+    if (ws_bad && tid == 0) atomicOr(err, kErrWs);
+  }
+}
+
 // ================================================================== warp-per-tile kernel
 
 __host__ __device__ inline int warp_slice_bytes(int G, int max_cand) {
@@ -1341,9 +1803,50 @@ int launch_warp(const AttendArgs &args, cudaStream_t stream) {
   return (int)cudaGetLastError();
 }
 
+template <int G, int CS, int RPH>
+int launch_lean_shape(const AttendArgs &a, cudaStream_t stream) {
+  const LeanLayout L = lean_layout(G, CS, a.max_cand);
+  auto kern = attend_lean_kernel<G, CS, RPH>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
+  if (e != cudaSuccess) return (int)e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(a.tiles * CS));
+  cfg.blockDim = dim3(kCtaThreads);
+  cfg.dynamicSmemBytes = (size_t)L.total;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, a);
+  if (e != cudaSuccess) return (int)e;
+  return (int)cudaGetLastError();
+}
+
+// The lean cluster kernel where its slices fit in registers; kNoLeanShape otherwise.
+constexpr int kNoLeanShape = -3;
+template <int G>
+int launch_lean(const AttendArgs &a, int CS, cudaStream_t stream) {
+  const int mc = a.max_cand;
+  if (mc > kLeanMaxCand) return kNoLeanShape;
+  if (CS == 4 && mc <= 4 * kHalfWarps * 2) return launch_lean_shape<G, 4, 2>(a, stream);
+  if constexpr (G <= 4) {
+    if (CS == 4 && mc <= 4 * kHalfWarps * 3) return launch_lean_shape<G, 4, 3>(a, stream);
+    if (CS == 2 && mc <= 2 * kHalfWarps * 4) return launch_lean_shape<G, 2, 4>(a, stream);
+  }
+  return kNoLeanShape;
+}
+
 template <int G>
 int launch_g(const AttendArgs &a, int kernel, int CS, cudaStream_t stream) {
   if (kernel == 2) return launch_warp<G>(a, stream);
+  if (kernel == 3) {
+    const int rc = launch_lean<G>(a, CS, stream);
+    if (rc != kNoLeanShape) return rc;
+  }
   switch (CS) {
     case 1: return launch_cta<G, 1>(a, stream);
     case 2: return launch_cta<G, 2>(a, stream);
@@ -1390,9 +1893,11 @@ int launch_attend(const AttendLaunch &l, void *stream) {
   a.tiles = l.geom.batch * l.geom.hkv * l.num_queries;
   const int sms = sm_count_cached();
   int kernel = l.kernel;
-  if (kernel == 0) kernel = (a.tiles <= sms) ? 1 : 2;  // CTA per tile while every tile has its own SM
+  // a cluster (or CTA) per tile while every tile has its own SM; the lean cluster kernel
+  // wherever its shape applies (launch_g falls back to the CTA kernel otherwise)
+  if (kernel == 0) kernel = (a.tiles <= sms) ? 3 : 2;
   int CS = l.cluster_size;
-  if (kernel == 1 && CS == 0) CS = (a.tiles * 4 <= sms) ? 4 : (a.tiles * 2 <= sms) ? 2 : 1;
+  if ((kernel == 1 || kernel == 3) && CS == 0) CS = (a.tiles * 4 <= sms) ? 4 : (a.tiles * 2 <= sms) ? 2 : 1;
   int rc;
   switch (l.group) {
     case 1: rc = launch_g<1>(a, kernel, CS, (cudaStream_t)stream); break;

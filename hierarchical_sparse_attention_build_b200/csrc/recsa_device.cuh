@@ -1,5 +1,5 @@
-// Device helpers for the sm_100a kernels: bf16 unpacking, shared-memory
-// mbarriers, bulk (TMA) global->shared row copies and bounded waits.
+// Device helpers for the sm_100a kernels: bf16 unpacking, order keys, the cluster
+// barrier and warp reductions.
 #pragma once
 
 #include <cstdint>
@@ -9,10 +9,6 @@
 #include "recsa_internal.h"
 
 namespace recsa {
-
-// Upper bound of any spin on an mbarrier: ~1.1 s at 1.9 GHz.  A wait that runs out
-// records kErrTimeout in the workspace error word and lets the kernel finish.
-constexpr long long kWaitCycles = 1ll << 31;
 
 __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
@@ -38,64 +34,11 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void fence_mbar_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Wait for the phase of `parity` to complete, at most kWaitCycles.  On timeout the
-// error word gets kErrTimeout and the caller proceeds (its data may be stale).
-// Once any wait of the launch has run out (the error word says so), later waits give
-// up at once, so a stuck copy costs one limit, not one per wait.
-__device__ __forceinline__ void mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *err) {
-  if (mbar_try_wait(bar, parity)) return;
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
-    if ((*reinterpret_cast<volatile uint32_t *>(err) & kErrTimeout) != 0u) return;
-    if (clock64() - t0 > kWaitCycles) {
-      atomicOr(err, kErrTimeout);
-      return;
-    }
-  }
-}
-
-// Bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from global
-// memory to this CTA's shared memory, completing on `bar` (transaction bytes).
-__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
 // Barrier over all threads of all CTAs of the cluster, with release/acquire ordering of
-// shared (and distributed shared) memory.
+// shared (and distributed shared) memory.  The .aligned form wants every lane of the
+// warp to execute it together, hence the warp sync in front.
 __device__ __forceinline__ void cluster_barrier() {
+  __syncwarp();
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 

@@ -118,8 +118,11 @@ typedef struct recsa_tree {
  *   entries  : int32 [tiles][2]; keys scored and values folded by the tile (rows read).
  *   kernel   : 0 = automatic; 1 = one CTA (or a cluster of cluster_size CTAs) per tile,
  *              the low-latency shape for few tiles; 2 = one warp per tile, the
- *              throughput shape for many tiles.  Results agree up to fp32 rounding.
- *   cluster_size: with kernel 1: 0 = automatic, or 1, 2, 4 CTAs per tile. */
+ *              throughput shape for many tiles; 3 = one cluster of 2 or 4 CTAs per
+ *              tile that exchanges scores by stores into its peers' shared memory
+ *              (one block barrier per level), where a level's candidates fit its
+ *              registers, else shape 1.  Results agree up to fp32 rounding.
+ *   cluster_size: with kernel 1 or 3: 0 = automatic, or 1, 2, 4 CTAs per tile. */
 typedef struct recsa_debug {
   int32_t *sel_idx;
   int32_t *entries;

@@ -38,8 +38,9 @@ def _compare_build(case: GpuCase, trees, b):
     return mism, total
 
 
-# launch shapes: (kernel, cluster_size); kernel 1 = CTA/cluster per tile, 2 = warp per tile
-SHAPES = [(1, 1), (1, 2), (1, 4), (2, 0)]
+# launch shapes: (kernel, cluster_size); kernel 1 = CTA/cluster per tile, 2 = warp per tile,
+# 3 = lean cluster per tile (score exchange by DSMEM stores)
+SHAPES = [(1, 1), (1, 2), (1, 4), (2, 0), (3, 2), (3, 4)]
 
 
 def _decode_and_check(case, trees, q, k, cluster_size=0, kernel=0):
@@ -155,7 +156,7 @@ def test_decode_k0_is_attention_over_top_summaries(kernel, cluster_size):
     (1, 2, 4, 3000, 5, 40, 1),     # many candidates per level (several gather chunks)
     (2, 1, 4, 2048, 4, 1, 4),      # k = 1
 ])
-@pytest.mark.parametrize("kernel,cluster_size", [(1, 1), (1, 4), (2, 0)])
+@pytest.mark.parametrize("kernel,cluster_size", [(1, 1), (1, 4), (2, 0), (3, 2), (3, 4)])
 def test_decode_odd_shapes(B, hkv, G, L, b, k, Q, kernel, cluster_size):
     inp = I.random_case(B, L, hkv, hkv * G, Q, seed=7 * L + b)
     case = GpuCase(inp, _params(hkv, G, b, k), L)
@@ -176,7 +177,7 @@ def test_decode_ties_keep_lower_index(kernel, cluster_size):
             assert lvl_sel == [0, 1, 2]
 
 
-@pytest.mark.parametrize("kernel", [1, 2])
+@pytest.mark.parametrize("kernel", [1, 2, 3])
 def test_decode_bf16_output_is_rounded_fp32_output(kernel):
     w = I.WORKLOADS["tiny_decode"]
     inp = I.decode_inputs(w)
