@@ -198,6 +198,33 @@ __device__ __forceinline__ Trig4 ldg_trig4(const float2 *table, int pos, int j16
   return r;
 }
 
+// The same row and table reads as ldg_row8 / ldg_trig4, issued where they stand: the
+// compiler keeps volatile asm in program order, so a level's rows go out before the
+// previous level is folded instead of being sunk next to their first use.
+__device__ __forceinline__ uint2 ld_nc_u2(const void *p) {
+  uint2 r;
+  asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+  return r;
+}
+__device__ __forceinline__ float4 ld_nc_f4(const void *p) {
+  float4 r;
+  asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w) : "l"(p));
+  return r;
+}
+__device__ __forceinline__ Row8 ld_row8_now(const uint16_t *row, int j16) {
+  Row8 r;
+  r.lo = ld_nc_u2(row + 4 * j16);
+  r.hi = ld_nc_u2(row + kHalf + 4 * j16);
+  return r;
+}
+__device__ __forceinline__ Trig4 ld_trig4_now(const float2 *table, int pos, int j16) {
+  const float4 *t = reinterpret_cast<const float4 *>(table + (int64_t)pos * kHalf + 4 * j16);
+  Trig4 r;
+  r.a = ld_nc_f4(t);
+  r.b = ld_nc_f4(t + 1);
+  return r;
+}
+
 __device__ __forceinline__ void unpack_row8(const Row8 &r, float (&lo)[4], float (&hi)[4]) {
   lo[0] = bf16_lo(r.lo.x);
   lo[1] = bf16_hi(r.lo.x);
@@ -1099,13 +1126,15 @@ __device__ __forceinline__ int count_above(const uint32_t *k, int j0, int j1, ui
   return cnt;
 }
 
-// Position of the e-th (0-based) set bit of the 256-bit mask w; e < popcount(w).
+// Position of the e-th (0-based) set bit of the mask w[0..NW) (32 bits a word);
+// e < popcount(w).
+template <int NW>
 __device__ __forceinline__ int nth_set(const uint32_t (&w)[8], int e) {
   int base = 0;
   uint32_t x = 0;
   bool found = false;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
+  for (int i = 0; i < NW; ++i) {
     const int c = __popc(w[i]);
     if (!found) {
       if (e < c) {
@@ -1212,9 +1241,9 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_lean_kernel(const Atten
     ok = valid && node >= 0 && node < lr.nrows;
     if (valid && !ok && j16 == 0) atomicOr(err, kErrIndex);
     if (ok) {
-      k = ldg_row8(lr.k + (int64_t)node * kD, j16);
-      v = ldg_row8(lr.v + (int64_t)node * kD, j16);
-      tr = ldg_trig4(a.table, pos, j16);
+      k = ld_row8_now(lr.k + (int64_t)node * kD, j16);
+      v = ld_row8_now(lr.v + (int64_t)node * kD, j16);
+      tr = ld_trig4_now(a.table, pos, j16);
     }
   };
   // node of candidate `pos` of the current level: the top level lists its nodes in
@@ -1335,26 +1364,51 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_lean_kernel(const Atten
         if (pos < hi) dst_kbuf[pb * kLeanMaxCand + pos] = key[r];
       }
     }
+    // the ranking reads whole chunks of 8: positions n .. n rounded up to 8 score nothing
+    if (tid < 8 && n + tid < ((n + 7) & ~7)) kbuf[pb * kLeanMaxCand + n + tid] = 0u;
+    const LevelRows lb = level_rows(a, geo, lvl - 1, t.bh);
     cluster_barrier();
 
     // 3. rank: candidate c is kept when fewer than top_k scorable candidates beat it
     //    (higher score, or equal score at a lower position)
+    uint32_t kw[8], ew[8];
     {
       const uint32_t *kb = kbuf + pb * kLeanMaxCand;
-      int c, j0, j1;
-      if (n <= 128) {  // two threads per candidate, half the competitors each
+      int c, better;
+      uint32_t kc;
+      if (n <= 128) {
+        // warp w ranks candidates 16w .. 16w+15 (lane j16), each half-warp taking half of
+        // every chunk of 8 competitors: half p reads positions 8t+4p .. 8t+4p+3 of chunk t.
+        // Chunks before 2w lie wholly below the warp's candidates (a tie there beats the
+        // candidate: count >=), chunks after 2w+1 wholly above (count >); only the two
+        // chunks of the warp's own candidates compare position by position.
         c = warp * 16 + j16;
-        const int h2 = (((n + 1) >> 1) + 3) & ~3;
-        j0 = min(n, (lane >> 4) * h2);
-        j1 = min(n, j0 + h2);
+        kc = c < n ? kb[c] : 0u;
+        const uint32_t thr_lo = kc - 1u, thr_hi = kc;
+        const int half4 = (lane >> 4) * 4, nch = (n + 7) >> 3, w0 = min(2 * warp, nch), w1 = min(2 * warp + 2, nch);
+        better = 0;
+#pragma unroll 4
+        for (int t8 = 0; t8 < w0; ++t8) {
+          const uint4 v = *reinterpret_cast<const uint4 *>(kb + 8 * t8 + half4);
+          better += (v.x > thr_lo) + (v.y > thr_lo) + (v.z > thr_lo) + (v.w > thr_lo);
+        }
+        for (int t8 = w0; t8 < w1; ++t8) {
+          const int j = 8 * t8 + half4;
+          const uint4 v = *reinterpret_cast<const uint4 *>(kb + j);
+          better += (v.x > (j < c ? thr_lo : thr_hi)) + (v.y > (j + 1 < c ? thr_lo : thr_hi)) +
+                    (v.z > (j + 2 < c ? thr_lo : thr_hi)) + (v.w > (j + 3 < c ? thr_lo : thr_hi));
+        }
+#pragma unroll 4
+        for (int t8 = w1; t8 < nch; ++t8) {
+          const uint4 v = *reinterpret_cast<const uint4 *>(kb + 8 * t8 + half4);
+          better += (v.x > thr_hi) + (v.y > thr_hi) + (v.z > thr_hi) + (v.w > thr_hi);
+        }
+        better += __shfl_xor_sync(F, better, 16);
       } else {
         c = tid;
-        j0 = 0;
-        j1 = n;
+        kc = c < n ? kb[c] : 0u;
+        better = count_above(kb, 0, min(n, c), kc - 1u) + count_above(kb, min(n, c + 1), n, kc);
       }
-      const uint32_t kc = c < n ? kb[c] : 0u;
-      int better = count_above(kb, j0, min(j1, max(j0, c)), kc - 1u) + count_above(kb, max(j0, min(j1, c + 1)), j1, kc);
-      if (n <= 128) better += __shfl_xor_sync(F, better, 16);
       const unsigned bal = __ballot_sync(F, c < n && kc != 0u && better < a.top_k);
       if (lane == 0) {
         uint16_t *mk = mask16 + pb * 16;
@@ -1367,7 +1421,6 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_lean_kernel(const Atten
       }
     }
     __syncthreads();
-    uint32_t kw[8], ew[8];
     {
       const uint4 w0 = *reinterpret_cast<const uint4 *>(mask16 + pb * 16);
       uint4 w1 = make_uint4(0u, 0u, 0u, 0u);
@@ -1385,7 +1438,13 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_lean_kernel(const Atten
     }
     values_read += m - min(a.top_k, m);
 
-    // 4. the next level: its size, forced node, this CTA's slice, and the slice's rows
+    // 4. the next level: this CTA's slice, the slice's rows, the level's size and forced
+    //    node.  Slices are cut from the expanded count alone: every CTA computes the same
+    //    cut, and together the slices cover every position (CS * 16 RPH >= max_cand), so
+    //    the row addresses need not wait for the last node's child count.
+    auto nth = [&](const uint32_t (&w)[8], int e) { return n <= 128 ? nth_set<4>(w, e) : nth_set<8>(w, e); };
+    const int per2 = min((nE * a.b + CS - 1) / CS, kHalfWarps * RPH);
+    const int lo2 = crank * per2;
     int n_next = 0, fpos_next = -1;
     if (last >= 0) {
       bool lf = false;
@@ -1399,27 +1458,23 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_lean_kernel(const Atten
       n_next = n_cap;
       if (fpos_next >= n_next) fpos_next = -1;
     }
-    const int per2 = (n_next + CS - 1) / CS;
-    const int lo2 = min(n_next, crank * per2), hi2 = min(n_next, lo2 + per2);
-    {
-      const LevelRows lb = level_rows(a, geo, lvl - 1, t.bh);
+    const int hi2 = min(n_next, lo2 + per2);
 #pragma unroll
-      for (int r = 0; r < RPH; ++r) {
-        const int i = lo2 + hw + kHalfWarps * r;
-        const bool valid = i < hi2 && i != fpos_next;
-        int node = 0;
-        if (valid) {
-          const int e = divb(i);
-          node = cand_node(par_cur, top, nth_set(ew, e)) * a.b + (i - e * a.b);
-        }
-        load_row(lb, i, node, valid, nk[r], nv[r], ntr[r], nok[r]);
+    for (int r = 0; r < RPH; ++r) {
+      const int i = lo2 + hw + kHalfWarps * r;
+      const bool valid = i < hi2 && i != fpos_next;
+      int node = 0;
+      if (valid) {
+        const int e = divb(i);
+        node = cand_node(par_cur, top, nth(ew, e)) * a.b + (i - e * a.b);
       }
-      ntq = ldg_trig4(a.table, n_next, j16);
+      load_row(lb, i, node, valid, nk[r], nv[r], ntr[r], nok[r]);
     }
-    if (tid < nE) par_all[(pb ^ 1) * MC + tid] = cand_node(par_cur, top, nth_set(ew, tid));
+    ntq = ld_trig4_now(a.table, n_next, j16);
+    if (tid < nE) par_all[(pb ^ 1) * MC + tid] = cand_node(par_cur, top, nth(ew, tid));
     if (a.sel_idx != nullptr && crank == 0 && lvl <= a.sel_levels) {
       int32_t *sel = a.sel_idx + ((int64_t)tile * a.sel_levels + (lvl - 1)) * a.top_k;
-      for (int u = tid; u < a.top_k; u += kCtaThreads) sel[u] = u < nK ? cand_node(par_cur, top, nth_set(kw, u)) : -1;
+      for (int u = tid; u < a.top_k; u += kCtaThreads) sel[u] = u < nK ? cand_node(par_cur, top, nth(kw, u)) : -1;
     }
 
     // 5. fold this level's unkept candidates while the next level's rows are in flight
