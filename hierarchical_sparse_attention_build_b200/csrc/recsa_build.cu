@@ -42,8 +42,9 @@ struct BuildArgs {
 
 // One CTA handles blocks of 64 nodes: each warp streams the children of 8 nodes
 // (lane = 4 consecutive dims, one 256-byte row per warp load), forms the child
-// means in fp32, writes the value rows, then the block applies W to the 64 key
-// means (W^T resident in shared memory, 8 nodes x 4 outputs per thread).
+// means in fp32, writes the value rows, then applies W to its own 8 key means (W^T
+// resident in shared memory, 8 nodes x 4 outputs per lane).  Warps share only W^T, so
+// they never wait for one another after it is loaded.
 __global__ void __launch_bounds__(kBuildThreads, 2) build_level_kernel(const BuildArgs a) {
   extern __shared__ __align__(16) float smem_f[];
   float *Wt = smem_f;               // Wt[k][o] = W[o][k]
@@ -71,7 +72,7 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_level_kernel(const Bui
         const uint16_t *kb = a.src_k + (a.src_row_off + bhi * a.src_slots) * kD + lane * 4;
         const uint16_t *vb = a.src_v + (a.src_row_off + bhi * a.src_slots) * kD + lane * 4;
         float wsum = 0.f;
-#pragma unroll 8
+#pragma unroll 16  // a whole node's children (b = 16) in flight at once
         for (int64_t c = c0; c < c1; ++c) {
           const uint2 ku = __ldg(reinterpret_cast<const uint2 *>(kb + c * kD));
           const uint2 vu = __ldg(reinterpret_cast<const uint2 *>(vb + c * kD));
@@ -99,7 +100,8 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_level_kernel(const Bui
       }
       *reinterpret_cast<float4 *>(Mean + nl * kD + lane * 4) = make_float4(ks[0], ks[1], ks[2], ks[3]);
     }
-    __syncthreads();
+    __syncwarp();  // a warp applies W to its own 8 nodes only: warps run out of step, so some
+                   // stream children while others compute
 
     // key = W @ mean for this warp's 8 nodes; lane owns outputs 4*lane .. 4*lane+3
     float acc[kNodesPerWarp][4];
@@ -136,7 +138,7 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_level_kernel(const Bui
         *reinterpret_cast<uint2 *>(a.dst_k + (a.dst_row_off + bhi * a.dst_slots + j) * kD + lane * 4) = ko;
       }
     }
-    __syncthreads();
+    __syncwarp();  // this warp's Mean rows are rewritten next
   }
 }
 
