@@ -71,23 +71,36 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_level_kernel(const Bui
         const int64_t c1 = min(c0 + (int64_t)a.b, a.n_prev);
         const uint16_t *kb = a.src_k + (a.src_row_off + bhi * a.src_slots) * kD + lane * 4;
         const uint16_t *vb = a.src_v + (a.src_row_off + bhi * a.src_slots) * kD + lane * 4;
-        float wsum = 0.f;
+        // Every child but the level's last covers span_prev tokens, so the value mean
+        // sums the children with weight 1 and then gives the last child, if it covers
+        // fewer tokens, its share f = tokens / span_prev.
 #pragma unroll 16  // a whole node's children (b = 16) in flight at once
         for (int64_t c = c0; c < c1; ++c) {
           const uint2 ku = __ldg(reinterpret_cast<const uint2 *>(kb + c * kD));
           const uint2 vu = __ldg(reinterpret_cast<const uint2 *>(vb + c * kD));
-          const float w = (float)min(a.span_prev, a.length - c * a.span_prev);
           ks[0] += bf16_lo(ku.x);
           ks[1] += bf16_hi(ku.x);
           ks[2] += bf16_lo(ku.y);
           ks[3] += bf16_hi(ku.y);
-          vs[0] += w * bf16_lo(vu.x);
-          vs[1] += w * bf16_hi(vu.x);
-          vs[2] += w * bf16_lo(vu.y);
-          vs[3] += w * bf16_hi(vu.y);
-          wsum += w;
+          vs[0] += bf16_lo(vu.x);
+          vs[1] += bf16_hi(vu.x);
+          vs[2] += bf16_lo(vu.y);
+          vs[3] += bf16_hi(vu.y);
         }
         const float nch = (float)(c1 - c0);
+        float wsum = nch;
+        if (c1 == a.n_prev && c1 > c0) {
+          const int64_t last_tokens = a.length - (c1 - 1) * a.span_prev;
+          if (last_tokens < a.span_prev) {
+            const float f1 = (float)last_tokens / (float)a.span_prev - 1.f;
+            const uint2 vu = __ldg(reinterpret_cast<const uint2 *>(vb + (c1 - 1) * kD));
+            vs[0] += f1 * bf16_lo(vu.x);
+            vs[1] += f1 * bf16_hi(vu.x);
+            vs[2] += f1 * bf16_lo(vu.y);
+            vs[3] += f1 * bf16_hi(vu.y);
+            wsum += f1;
+          }
+        }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           ks[i] = ks[i] / nch;
