@@ -257,3 +257,42 @@ def test_prefill_then_decode():
     kc, vc = O.append_chunk(bits(inp["k_tok"]), bits(inp["v_tok"]), bits(inp["k_new"]), bits(inp["v_new"]), L)
     trees = O.build_all(kc, vc, inp["pooler"].double().numpy(), b, L + C)
     _decode_and_check(case, trees, q, k)
+
+
+def test_token_by_token_decode_loop():
+    """A decode loop: each step appends one token (chunk of 1) and attends its query, so the
+    tree is extended by one node per level per step; the steps cross 1024 = 4^5 tokens, where
+    a new top level appears.  Every step against the oracle, then the node rows against a
+    fresh build over all tokens."""
+    L, S, b, k, hkv, G = 1021, 6, 4, 2, 2, 4
+    inp = I.random_case(1, L, hkv, hkv * G, 1, seed=33, capacity=L + S, chunk=S)
+    case = GpuCase(inp, _params(hkv, G, b, k), L)
+    case.build()
+    kc, vc = bits(inp["k_tok"]), bits(inp["v_tok"])
+    pooler = inp["pooler"].double().numpy()
+    stats = Stats()
+    for s in range(S):
+        kn, vn, qs = (inp[x][:, s:s + 1].contiguous() for x in ("k_new", "v_new", "q"))
+        out, sel, ent = case.prefill(kn, vn, qs)
+        assert case.tree.length == L + s + 1
+        kc, vc = O.append_chunk(kc, vc, bits(kn), bits(vn), L + s)
+        trees = O.build_all(kc, vc, pooler, b, L + s + 1)
+        p = L + s
+        top = len(O.level_counts(p, b)) - 1
+        qb = bits(qs)
+        for h in range(hkv):
+            check_tile(stats, O.bf16_bits_to_f64(qb[0, 0, h * G:(h + 1) * G]), trees[0][h], p, k, True,
+                       out[0, 0, h * G:(h + 1) * G].numpy(), gpu_selection(sel, h, top), ent[h])
+    stats.assert_ok()
+    mism = total = 0
+    for lvl in range(1, trees[0][0].top + 1):
+        gk, gv = case.node_bits(lvl)
+        for h in range(hkv):
+            t = trees[0][h]
+            n = t.keys[lvl].shape[0]
+            for got, want in ((gk[0, h, :n], t.keys[lvl]), (gv[0, h, :n], t.values[lvl])):
+                m, c = check_node_rows(got, want)
+                mism += m
+                total += c
+    assert mism <= total * 1e-2
+    print("decode loop", stats)
