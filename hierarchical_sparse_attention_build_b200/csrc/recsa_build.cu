@@ -63,6 +63,8 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_level_kernel(const Bui
     for (int t = 0; t < kNodesPerWarp; ++t) {
       const int nl = warp * kNodesPerWarp + t;
       const int64_t id = base + nl;
+      float2 ks2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // dims (0,1), (2,3) of the lane's 4
+      float2 vs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       float ks[4] = {0.f, 0.f, 0.f, 0.f}, vs[4] = {0.f, 0.f, 0.f, 0.f};
       if (id < total) {
         const int64_t bhi = id / a.nj;
@@ -78,15 +80,13 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_level_kernel(const Bui
         for (int64_t c = c0; c < c1; ++c) {
           const uint2 ku = __ldg(reinterpret_cast<const uint2 *>(kb + c * kD));
           const uint2 vu = __ldg(reinterpret_cast<const uint2 *>(vb + c * kD));
-          ks[0] += bf16_lo(ku.x);
-          ks[1] += bf16_hi(ku.x);
-          ks[2] += bf16_lo(ku.y);
-          ks[3] += bf16_hi(ku.y);
-          vs[0] += bf16_lo(vu.x);
-          vs[1] += bf16_hi(vu.x);
-          vs[2] += bf16_lo(vu.y);
-          vs[3] += bf16_hi(vu.y);
+          ks2[0] = __fadd2_rn(ks2[0], make_float2(bf16_lo(ku.x), bf16_hi(ku.x)));
+          ks2[1] = __fadd2_rn(ks2[1], make_float2(bf16_lo(ku.y), bf16_hi(ku.y)));
+          vs2[0] = __fadd2_rn(vs2[0], make_float2(bf16_lo(vu.x), bf16_hi(vu.x)));
+          vs2[1] = __fadd2_rn(vs2[1], make_float2(bf16_lo(vu.y), bf16_hi(vu.y)));
         }
+        ks[0] = ks2[0].x, ks[1] = ks2[0].y, ks[2] = ks2[1].x, ks[3] = ks2[1].y;
+        vs[0] = vs2[0].x, vs[1] = vs2[0].y, vs[2] = vs2[1].x, vs[3] = vs2[1].y;
         const float nch = (float)(c1 - c0);
         float wsum = nch;
         if (c1 == a.n_prev && c1 > c0) {
@@ -116,28 +116,41 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_level_kernel(const Bui
     __syncwarp();  // a warp applies W to its own 8 nodes only: warps run out of step, so some
                    // stream children while others compute
 
-    // key = W @ mean for this warp's 8 nodes; lane owns outputs 4*lane .. 4*lane+3
-    float acc[kNodesPerWarp][4];
+    // key = W @ mean for this warp's 8 nodes; lane owns outputs 4*lane .. 4*lane+3, as the
+    // pairs (4l, 4l+1) and (4l+2, 4l+3) of packed fp32 FMAs (each output's terms in k order)
+    float2 acc2[kNodesPerWarp][2];
 #pragma unroll
-    for (int n = 0; n < kNodesPerWarp; ++n)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
+    for (int n = 0; n < kNodesPerWarp; ++n) acc2[n][0] = acc2[n][1] = make_float2(0.f, 0.f);
     const float4 *Wt4 = reinterpret_cast<const float4 *>(Wt);
     const float4 *M4 = reinterpret_cast<const float4 *>(Mean);
 #pragma unroll 2
     for (int k = 0; k < kD; k += 4) {
-      const float4 w0 = Wt4[(k + 0) * 32 + lane];
-      const float4 w1 = Wt4[(k + 1) * 32 + lane];
-      const float4 w2 = Wt4[(k + 2) * 32 + lane];
-      const float4 w3 = Wt4[(k + 3) * 32 + lane];
+      float2 w[4][2];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float4 wt = Wt4[(k + t) * 32 + lane];
+        w[t][0] = make_float2(wt.x, wt.y);
+        w[t][1] = make_float2(wt.z, wt.w);
+      }
 #pragma unroll
       for (int n = 0; n < kNodesPerWarp; ++n) {
         const float4 m = M4[(warp * kNodesPerWarp + n) * 32 + (k >> 2)];
-        acc[n][0] = fmaf(m.w, w3.x, fmaf(m.z, w2.x, fmaf(m.y, w1.x, fmaf(m.x, w0.x, acc[n][0]))));
-        acc[n][1] = fmaf(m.w, w3.y, fmaf(m.z, w2.y, fmaf(m.y, w1.y, fmaf(m.x, w0.y, acc[n][1]))));
-        acc[n][2] = fmaf(m.w, w3.z, fmaf(m.z, w2.z, fmaf(m.y, w1.z, fmaf(m.x, w0.z, acc[n][2]))));
-        acc[n][3] = fmaf(m.w, w3.w, fmaf(m.z, w2.w, fmaf(m.y, w1.w, fmaf(m.x, w0.w, acc[n][3]))));
+        const float mt[4] = {m.x, m.y, m.z, m.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float2 mm = make_float2(mt[t], mt[t]);
+          acc2[n][0] = __ffma2_rn(mm, w[t][0], acc2[n][0]);
+          acc2[n][1] = __ffma2_rn(mm, w[t][1], acc2[n][1]);
+        }
       }
+    }
+    float acc[kNodesPerWarp][4];
+#pragma unroll
+    for (int n = 0; n < kNodesPerWarp; ++n) {
+      acc[n][0] = acc2[n][0].x;
+      acc[n][1] = acc2[n][0].y;
+      acc[n][2] = acc2[n][1].x;
+      acc[n][3] = acc2[n][1].y;
     }
 #pragma unroll
     for (int n = 0; n < kNodesPerWarp; ++n) {
