@@ -272,11 +272,16 @@ __device__ __forceinline__ void rotated_query(const float *qraw, const Trig4 &tq
 template <int G>
 __device__ __forceinline__ void dot_row8(const Row8 &k, const Trig4 &tr, const float2 (&q2lo)[G][2],
                                          const float2 (&q2hi)[G][2], float (&part)[G]) {
-  float lo[4], hi[4];
-  unpack_row8(k, lo, hi);
-  rotate4(lo, hi, tr);
-  const float2 l01 = make_float2(lo[0], lo[1]), l23 = make_float2(lo[2], lo[3]);
-  const float2 h01 = make_float2(hi[0], hi[1]), h23 = make_float2(hi[2], hi[3]);
+  // the key's RoPE pairs rotated two at a time (packed fp32): lo' = lo c - hi s,
+  // hi' = hi c + lo s, with (c, c') and (s, s') straight from the table
+  const float2 k01 = make_float2(bf16_lo(k.lo.x), bf16_hi(k.lo.x)), k23 = make_float2(bf16_lo(k.lo.y), bf16_hi(k.lo.y));
+  const float2 g01 = make_float2(bf16_lo(k.hi.x), bf16_hi(k.hi.x)), g23 = make_float2(bf16_lo(k.hi.y), bf16_hi(k.hi.y));
+  const float2 c01 = make_float2(tr.a.x, tr.a.y), s01 = make_float2(tr.a.z, tr.a.w);
+  const float2 c23 = make_float2(tr.b.x, tr.b.y), s23 = make_float2(tr.b.z, tr.b.w);
+  const float2 l01 = __ffma2_rn(k01, c01, __fmul2_rn(g01, make_float2(-s01.x, -s01.y)));
+  const float2 l23 = __ffma2_rn(k23, c23, __fmul2_rn(g23, make_float2(-s23.x, -s23.y)));
+  const float2 h01 = __ffma2_rn(g01, c01, __fmul2_rn(k01, s01));
+  const float2 h23 = __ffma2_rn(g23, c23, __fmul2_rn(k23, s23));
 #pragma unroll
   for (int h = 0; h < G; ++h) {
     float2 x = __fmul2_rn(q2lo[h][0], l01);
