@@ -54,9 +54,12 @@ struct TBarrier {
     name = std::move(nm);
   }
   void wait(int line);
+  long arrive(int line);             // split form: returns the generation to wait for
+  void wait_gen(long my, int line);
 };
 
 extern thread_local int t_tid, t_block, t_crank, t_cs;
+extern thread_local long t_cluster_gen;  // cluster-barrier generation this thread arrived at
 extern thread_local unsigned char *t_smem;
 extern std::vector<unsigned char *> g_cluster_smem;  // per cluster rank
 extern size_t g_smem_bytes;
@@ -84,6 +87,31 @@ inline void TBarrier::wait(int line) {
     char buf[256];
     snprintf(buf, sizeof buf, "barrier '%s' at line %d timed out (%d of %d arrived)", name.c_str(), line, arrived,
              count);
+    report_and_abort(buf);
+  }
+}
+
+inline long TBarrier::arrive(int line) {
+  g_where[t_crank * 256 + t_tid].line = line;
+  g_where[t_crank * 256 + t_tid].what = "cluster-arrive";
+  std::lock_guard<std::mutex> lk(mu);
+  const long my = gen;
+  if (++arrived == count) {
+    arrived = 0;
+    ++gen;
+    cv.notify_all();
+  }
+  return my;
+}
+
+inline void TBarrier::wait_gen(long my, int line) {
+  g_where[t_crank * 256 + t_tid].line = line;
+  g_where[t_crank * 256 + t_tid].what = name.c_str();
+  std::unique_lock<std::mutex> lk(mu);
+  if (!cv.wait_for(lk, std::chrono::seconds(20), [&] { return gen != my; })) {
+    lk.unlock();
+    char buf[256];
+    snprintf(buf, sizeof buf, "barrier '%s' (split wait) at line %d timed out", name.c_str(), line);
     report_and_abort(buf);
   }
 }

@@ -18,4 +18,8 @@ inline uint32_t order_key(float f) {
 }
 #define cluster_barrier() \
   do { __syncwarp(); emu::g_cluster_bar.wait(__LINE__); } while (0)
+#define cluster_arrive() \
+  do { emu::t_cluster_gen = emu::g_cluster_bar.arrive(__LINE__); } while (0)
+#define cluster_wait() \
+  do { emu::g_cluster_bar.wait_gen(emu::t_cluster_gen, __LINE__); } while (0)
 }  // namespace recsa
