@@ -1953,9 +1953,12 @@ int launch_attend(const AttendLaunch &l, void *stream) {
   a.tiles = l.geom.batch * l.geom.hkv * l.num_queries;
   const int sms = sm_count_cached();
   int kernel = l.kernel;
-  // a cluster (or CTA) per tile while every tile has its own SM; the lean cluster kernel
-  // wherever its shape applies (launch_g falls back to the CTA kernel otherwise)
-  if (kernel == 0) kernel = (a.tiles <= sms) ? 3 : 2;
+  // A cluster (or CTA) per tile while every tile has its own SM, the lean cluster kernel
+  // wherever its shape applies (launch_g falls back to the CTA kernel otherwise).  Up to
+  // 4 waves of tiles a CTA per tile still finishes first: a wave costs about a fifth of
+  // what one warp takes to walk a tile alone, and the warp-per-tile grid holds every tile
+  // at once only beyond that.
+  if (kernel == 0) kernel = (a.tiles <= sms) ? 3 : (a.tiles <= 4 * sms) ? 1 : 2;
   int CS = l.cluster_size;
   if ((kernel == 1 || kernel == 3) && CS == 0) CS = (a.tiles * 4 <= sms) ? 4 : (a.tiles * 2 <= sms) ? 2 : 1;
   int rc;
