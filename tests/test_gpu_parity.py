@@ -296,3 +296,11 @@ def test_token_by_token_decode_loop():
                 total += c
     assert mism <= total * 1e-2
     print("decode loop", stats)
+
+
+def test_prefill_levels_past_128_candidates():
+    # causal, b = 16, k = 8: a level holds up to (k + 1) b = 144 candidates, so the cluster
+    # kernel takes 3 rows per half-warp and ranks by the generic count (24 tiles: automatic
+    # launch picks 4-CTA clusters)
+    stats, _ = _prefill_check(1, 1, 4, 3000, 24, 16, 8, seed=5)
+    print("prefill 144 candidates", stats)

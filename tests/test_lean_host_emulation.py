@@ -152,3 +152,9 @@ def test_decode_matches_oracle(emu_bin, tmp_path, B, hkv, G, L, b, k, Q, CS):
 @pytest.mark.parametrize("CS", [2, 4])
 def test_causal_prefill_matches_oracle(emu_bin, tmp_path, CS):
     _run(emu_bin, tmp_path, 1, 1, 4, 200, 4, 2, 6, CS, causal=True)
+
+
+def test_causal_levels_past_128_candidates(emu_bin, tmp_path):
+    # b = 16, k = 8, causal: up to 144 candidates a level, 3 rows per half-warp, and the
+    # ranking by the generic count
+    _run(emu_bin, tmp_path, 1, 1, 4, 3000, 16, 8, 6, 4, causal=True, seed=5)
