@@ -94,6 +94,7 @@ def _load() -> ctypes.CDLL:
         "recsa_workspace_init": [P, i64, vp, sz, vp],
         "recsa_build_tree": [P, T, vp],
         "recsa_decode": [P, T, vp, i32, vp, i32, vp, sz, D, vp],
+        "recsa_decode_host": [P, T, vp, i32, vp, i32, vp, vp, vp, sz, D, vp],
         "recsa_prefill_chunk": [P, T, vp, vp, vp, i32, vp, i32, vp, sz, D, vp],
         "recsa_check_device_errors": [vp, vp],
         "recsa_decode_no_alloc": [P, T, vp, i32, vp, i32, vp],
@@ -225,6 +226,18 @@ def decode(p: Params, tree: RecsaTree, q: torch.Tensor, out: torch.Tensor, ws: W
     _check(_lib.recsa_decode(ctypes.byref(p), ctypes.byref(tree.c), _ptr(q), nq, _ptr(out),
                              int(out.dtype == torch.float32), _ptr(ws.buf), ws.nbytes,
                              ctypes.byref(dbg) if dbg is not None else None, _stream(stream)))
+
+
+def decode_host(p: Params, tree: RecsaTree, q_host: torch.Tensor, out_host: torch.Tensor, q_dev: torch.Tensor,
+                out_dev: torch.Tensor, ws: Workspace, stream=None) -> None:
+    """recsa_decode_host: host q -> device staging -> decode -> host out, queued in one call."""
+    for t in (q_host, out_host):
+        assert t.device.type == "cpu" and t.is_contiguous()
+    assert q_host.dtype == torch.bfloat16 and q_dev.shape == q_host.shape and out_dev.shape == out_host.shape
+    assert out_dev.dtype == out_host.dtype and q_dev.is_contiguous() and out_dev.is_contiguous()
+    _check(_lib.recsa_decode_host(ctypes.byref(p), ctypes.byref(tree.c), _ptr(q_host), q_host.shape[1],
+                                  _ptr(out_host), int(out_host.dtype == torch.float32), _ptr(q_dev), _ptr(out_dev),
+                                  _ptr(ws.buf), ws.nbytes, None, _stream(stream)))
 
 
 def prefill_chunk(p: Params, tree: RecsaTree, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor,

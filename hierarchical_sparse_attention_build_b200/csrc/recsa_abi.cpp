@@ -175,6 +175,48 @@ recsa_status build_range(const TreeGeom &g, const recsa_tree &t, int64_t length,
   return RECSA_OK;
 }
 
+// Every check of a decode call and the launch it becomes (nothing is queued here).
+recsa_status decode_launch(const recsa_params *params, const recsa_tree *tree, const void *q, int32_t num_queries,
+                           void *out, int32_t out_is_fp32, void *ws, size_t ws_bytes, const recsa_debug *debug,
+                           AttendLaunch *l) {
+  recsa_status s = check_params(params);
+  if (s != RECSA_OK) return s;
+  TreeGeom g;
+  s = check_tree(params, tree, &g);
+  if (s != RECSA_OK) return s;
+  if (tree->length < 1) return fail(RECSA_ERR_INVALID_ARGUMENT, "decode needs length >= 1");
+  if (num_queries < 1) return fail(RECSA_ERR_INVALID_ARGUMENT, "num_queries %d < 1", num_queries);
+  if (!q || !out) return fail(RECSA_ERR_INVALID_ARGUMENT, "q or out is NULL");
+  if (!aligned16(q) || !aligned16(out)) return fail(RECSA_ERR_INVALID_ARGUMENT, "q or out is not 16-byte aligned");
+  s = check_ws(params, tree, ws, ws_bytes);
+  if (s != RECSA_OK) return s;
+  s = check_debug(params, debug);
+  if (s != RECSA_OK) return s;
+  const int64_t mc = max_candidates(params, tree->length, false);
+  if (mc > kMaxCand)
+    return fail(RECSA_ERR_UNSUPPORTED, "up to %lld candidates per level > %d", (long long)mc, kMaxCand);
+  const int64_t tiles = (int64_t)tree->batch * params->num_kv_heads * num_queries;
+  if (tiles > 0x7fffffff / 4) return fail(RECSA_ERR_UNSUPPORTED, "%lld tiles", (long long)tiles);
+  l->geom = g;
+  l->tree = *tree;
+  l->q = q;
+  l->out = out;
+  l->out_fp32 = out_is_fp32 ? 1 : 0;
+  l->num_queries = num_queries;
+  l->length = tree->length;
+  l->causal = 0;
+  l->group = params->num_q_heads / params->num_kv_heads;
+  l->top_k = params->top_k;
+  l->scale = params->softmax_scale > 0.f ? params->softmax_scale : 1.0f / std::sqrt((float)kD);
+  l->ws = ws;
+  l->table_rows_needed = (int)mc + 1;
+  l->max_cand = (int)((mc + 31) / 32 * 32);
+  l->cluster_size = debug ? debug->cluster_size : 0;
+  l->kernel = debug ? debug->kernel : 0;
+  l->debug = debug;
+  return RECSA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -246,44 +288,50 @@ RECSA_API recsa_status recsa_build_tree(const recsa_params *params, const recsa_
 RECSA_API recsa_status recsa_decode(const recsa_params *params, const recsa_tree *tree, const void *q,
                                     int32_t num_queries, void *out, int32_t out_is_fp32, void *ws, size_t ws_bytes,
                                     const recsa_debug *debug, recsa_stream_t stream) {
-  recsa_status s = check_params(params);
-  if (s != RECSA_OK) return s;
-  TreeGeom g;
-  s = check_tree(params, tree, &g);
-  if (s != RECSA_OK) return s;
-  if (tree->length < 1) return fail(RECSA_ERR_INVALID_ARGUMENT, "decode needs length >= 1");
-  if (num_queries < 1) return fail(RECSA_ERR_INVALID_ARGUMENT, "num_queries %d < 1", num_queries);
-  if (!q || !out) return fail(RECSA_ERR_INVALID_ARGUMENT, "q or out is NULL");
-  if (!aligned16(q) || !aligned16(out)) return fail(RECSA_ERR_INVALID_ARGUMENT, "q or out is not 16-byte aligned");
-  s = check_ws(params, tree, ws, ws_bytes);
-  if (s != RECSA_OK) return s;
-  s = check_debug(params, debug);
-  if (s != RECSA_OK) return s;
-  const int64_t mc = max_candidates(params, tree->length, false);
-  if (mc > kMaxCand)
-    return fail(RECSA_ERR_UNSUPPORTED, "up to %lld candidates per level > %d", (long long)mc, kMaxCand);
-  const int64_t tiles = (int64_t)tree->batch * params->num_kv_heads * num_queries;
-  if (tiles > 0x7fffffff / 4) return fail(RECSA_ERR_UNSUPPORTED, "%lld tiles", (long long)tiles);
   AttendLaunch l;
-  l.geom = g;
-  l.tree = *tree;
-  l.q = q;
-  l.out = out;
-  l.out_fp32 = out_is_fp32 ? 1 : 0;
-  l.num_queries = num_queries;
-  l.length = tree->length;
-  l.causal = 0;
-  l.group = params->num_q_heads / params->num_kv_heads;
-  l.top_k = params->top_k;
-  l.scale = params->softmax_scale > 0.f ? params->softmax_scale : 1.0f / std::sqrt((float)kD);
-  l.ws = ws;
-  l.table_rows_needed = (int)mc + 1;
-  l.max_cand = (int)((mc + 31) / 32 * 32);
-  l.cluster_size = debug ? debug->cluster_size : 0;
-  l.kernel = debug ? debug->kernel : 0;
-  l.debug = debug;
+  const recsa_status s = decode_launch(params, tree, q, num_queries, out, out_is_fp32, ws, ws_bytes, debug, &l);
+  if (s != RECSA_OK) return s;
   const int rc = launch_attend(l, stream);
   if (rc != 0) return cuda_fail(rc, "decode attend");
+  return RECSA_OK;
+}
+
+RECSA_API recsa_status recsa_decode_host(const recsa_params *params, const recsa_tree *tree, const void *q_host,
+                                         int32_t num_queries, void *out_host, int32_t out_is_fp32, void *q_dev,
+                                         void *out_dev, void *ws, size_t ws_bytes, const recsa_debug *debug,
+                                         recsa_stream_t stream) {
+  if (!q_host || !out_host) return fail(RECSA_ERR_INVALID_ARGUMENT, "q_host or out_host is NULL");
+  if (!aligned16(q_host) || !aligned16(out_host))
+    return fail(RECSA_ERR_INVALID_ARGUMENT, "q_host or out_host is not 16-byte aligned");
+  AttendLaunch l;  // every check, on the staging buffers, before any CUDA call
+  const recsa_status s = decode_launch(params, tree, q_dev, num_queries, out_dev, out_is_fp32, ws, ws_bytes, debug, &l);
+  if (s != RECSA_OK) return s;
+  // Pinned host memory is mapped into the device's address space: the kernel then reads
+  // the queries and writes the outputs across the host link itself (no staging copy).
+  // Pageable memory goes through the staging buffers.
+  auto mapped = [](const void *host) -> void * {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, host) != cudaSuccess) {
+      cudaGetLastError();  // a pointer the runtime does not know: not an error of this call
+      return nullptr;
+    }
+    return at.type == cudaMemoryTypeHost ? at.devicePointer : nullptr;
+  };
+  void *q_map = mapped(q_host), *out_map = mapped(out_host);
+  if (q_map) l.q = q_map;
+  if (out_map) l.out = out_map;
+  const size_t q_bytes = (size_t)tree->batch * num_queries * params->num_q_heads * kD * 2;
+  const size_t out_bytes = q_bytes * (out_is_fp32 ? 2 : 1);
+  if (!q_map) {
+    const cudaError_t e = cudaMemcpyAsync(q_dev, q_host, q_bytes, cudaMemcpyHostToDevice, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail((int)e, "copy of the queries to the device");
+  }
+  const int rc = launch_attend(l, stream);
+  if (rc != 0) return cuda_fail(rc, "decode attend");
+  if (!out_map) {
+    const cudaError_t e = cudaMemcpyAsync(out_host, out_dev, out_bytes, cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail((int)e, "copy of the output to the host");
+  }
   return RECSA_OK;
 }
 

@@ -172,6 +172,24 @@ RECSA_API recsa_status recsa_decode(const recsa_params *params, const recsa_tree
                                     int32_t num_queries, void *out, int32_t out_is_fp32, void *ws,
                                     size_t ws_bytes, const recsa_debug *debug, recsa_stream_t stream);
 
+/* recsa_decode on host buffers: one call takes a batch of queries in host memory to
+ * attention outputs in host memory, queued on `stream`.  A pinned (page-locked) host
+ * buffer is read or written by the decode kernel itself through its device mapping; a
+ * pageable one is copied through the staging buffer (q_host -> q_dev before the decode,
+ * out_dev -> out_host after it).  Not in the abstract: the plumbing a host-side caller
+ * needs around recsa_decode.
+ *   q_host   : host bf16 [batch][num_queries][Hq][128], 16-byte aligned.
+ *   out_host : host output of the same shape, fp32 if out_is_fp32 else bf16, 16-byte aligned.
+ *   q_dev, out_dev : device staging buffers of those sizes (16-byte aligned), owned by the
+ *              caller (untouched when the host buffer is pinned).
+ * The host buffers must stay untouched until the stream passes this call (out_host holds
+ * the result after that).  Every argument is checked, as recsa_decode checks its own,
+ * before anything is queued; a failed copy returns RECSA_ERR_CUDA. */
+RECSA_API recsa_status recsa_decode_host(const recsa_params *params, const recsa_tree *tree, const void *q_host,
+                                         int32_t num_queries, void *out_host, int32_t out_is_fp32, void *q_dev,
+                                         void *out_dev, void *ws, size_t ws_bytes, const recsa_debug *debug,
+                                         recsa_stream_t stream);
+
 /* Causal prefill of a chunk of `chunk` tokens at positions L .. L+chunk-1
  * (L = tree->length): appends k_new / v_new to the token caches, rebuilds the tree
  * nodes those tokens touch (and any level that becomes new), then attends query i

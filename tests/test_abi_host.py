@@ -29,7 +29,7 @@ def test_library_exports_every_declared_symbol():
     names = declared_functions()
     assert set(names) == {"recsa_tree_layout", "recsa_workspace_size", "recsa_workspace_init", "recsa_build_tree",
                           "recsa_decode", "recsa_prefill_chunk", "recsa_check_device_errors", "recsa_status_string",
-                          "recsa_last_error", "recsa_decode_no_alloc"}, names
+                          "recsa_last_error", "recsa_decode_no_alloc", "recsa_decode_host"}, names
     for n in names:
         assert hasattr(lib, n), n
         assert ctypes.cast(getattr(lib, n), ctypes.c_void_p).value
@@ -109,6 +109,25 @@ def _decode(p, t, q=FAKE, nq=1, out=FAKE, ws=FAKE, ws_bytes=1 << 30, dbg=None):
 ])
 def test_decode_bad_tree_rejected(tkw, code):
     assert _decode(_p(), _tree(**tkw)) == code
+
+
+def test_decode_host_checks_everything_before_queuing():
+    # each of these fails validation, so no copy is queued and no CUDA call is made
+    p, t = _p(), _tree()
+    host = ctypes.create_string_buffer(64)
+
+    def call(q_host=host, out_host=host, q_dev=FAKE, out_dev=FAKE, ws_bytes=1 << 30, p=p, t=t, nq=1):
+        return lib.recsa_decode_host(ctypes.byref(p), ctypes.byref(t), q_host, nq, out_host, 1, q_dev, out_dev,
+                                     FAKE, ws_bytes, None, None)
+
+    assert call(q_host=None) == INVALID
+    assert call(out_host=None) == INVALID
+    assert call(q_dev=0) == INVALID
+    assert call(out_dev=FAKE + 8) == INVALID
+    assert call(nq=0) == INVALID
+    assert call(ws_bytes=100) == WS_SMALL
+    assert call(p=_p(num_q_heads=30)) == INVALID
+    assert call(t=_tree(length=0)) == INVALID
 
 
 def test_decode_bad_call_arguments_rejected():

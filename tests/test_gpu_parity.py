@@ -304,3 +304,31 @@ def test_prefill_levels_past_128_candidates():
     # launch picks 4-CTA clusters)
     stats, _ = _prefill_check(1, 1, 4, 3000, 24, 16, 8, seed=5)
     print("prefill 144 candidates", stats)
+
+
+@pytest.mark.parametrize("pinned", [True, False])
+def test_decode_from_host_buffers_equals_decode(pinned):
+    """recsa_decode_host: host queries in, host outputs back, one call; the same results as
+    recsa_decode on device buffers (fp32 and bf16 outputs).  Pinned buffers are read and
+    written by the kernel through their device mapping, pageable ones through the staging
+    buffers."""
+    w = I.WORKLOADS["tiny_decode"]
+    inp = I.decode_inputs(w, device="cpu")
+    case = GpuCase(inp, _params(w.kv_heads, w.q_heads // w.kv_heads, w.branching, w.top_k), w.length)
+    case.build()
+    q = inp["q"].contiguous()
+    for dtype in (torch.float32, torch.bfloat16):
+        out_ref = torch.empty(q.shape, dtype=dtype, device="cuda")
+        R.decode(case.p, case.tree, q.cuda(), out_ref, case.ws)
+        q_host = q.clone()
+        out_host = torch.full(q.shape, -3.0, dtype=dtype)
+        if pinned:
+            q_host, out_host = q_host.pin_memory(), out_host.pin_memory()
+        q_dev = torch.zeros(q.shape, dtype=torch.bfloat16, device="cuda")
+        out_dev = torch.zeros(q.shape, dtype=dtype, device="cuda")
+        R.decode_host(case.p, case.tree, q_host, out_host, q_dev, out_dev, case.ws)
+        torch.cuda.synchronize()
+        R.check_device_errors(case.ws)
+        assert torch.equal(out_host, out_ref.cpu())
+        # the staging buffers are used exactly when the host buffers are pageable
+        assert (torch.count_nonzero(out_dev).item() == 0) == pinned
