@@ -291,6 +291,41 @@ def leg_prefill(R, timer, args, dist_on, hbm_peak, name, length):
                     "queries hit L2, so logical GB/s can exceed HBM bandwidth"}
 
 
+def leg_decode_loop(R, timer, args, dist_on):
+    """Token-by-token decode at 1M (B = 4): every step appends one token to each sequence
+    (its K and V), extends the tree over it and attends that token's query, i.e.
+    recsa_prefill_chunk with a chunk of 1 -- the step a decode loop runs per token."""
+    w = I.WORKLOADS["decode_1m"]
+    warmup, steps = 4, 64 if not args.quick else 16
+    inp = I.decode_inputs(w, device="cuda", capacity=w.length + warmup + steps + 8)
+    p = R.params(num_kv_heads=w.kv_heads, num_q_heads=w.q_heads, branching=w.branching, top_k=w.top_k)
+    tree, ws = make_tree(R, p, inp, w.length)
+    g = torch.Generator(device="cuda").manual_seed(91)
+    B, Hkv, Hq = w.batch, w.kv_heads, w.q_heads
+    toks = [tuple(torch.randn(B, 1, h, 128, generator=g, device="cuda").to(torch.bfloat16) for h in (Hkv, Hkv, Hq))
+            for _ in range(warmup + steps + 1)]
+    out = torch.empty(B, 1, Hq, 128, dtype=torch.bfloat16, device="cuda")
+    nxt = [0]
+
+    def step():
+        kn, vn, qn = toks[nxt[0]]
+        nxt[0] += 1
+        R.prefill_chunk(p, tree, kn, vn, qn, out, ws)
+
+    per, _ = timer.run(step, steps, warmup)
+    t = max_over_ranks(sum(per), dist_on) / steps
+    R.check_device_errors(ws)
+    levels = tree.levels
+    del tree, ws, inp
+    torch.cuda.empty_cache()
+    return {"workload": f"decode_loop_1m: B={B}, L={w.length} + 1 token per sequence per step, Hq={Hq}, "
+                        f"Hkv={Hkv}, b={w.branching}, k={w.top_k}",
+            "tokens_per_s": B / t, "us_per_step": t * 1e6,
+            "launches_per_step": 2 + levels,
+            "note": "append + the tree extension (one node per level per head) + causal attend of the new "
+                    "token; each step grows the cache by one token"}
+
+
 def leg_build_2m(R, timer, args, dist_on, hbm_peak):
     w = I.WORKLOADS["build_decode_2m"]
     inp = I.decode_inputs(w, device="cuda")
@@ -474,6 +509,7 @@ def run_gpu(args):
         extra["prefill"] = leg_prefill(R, timer, args, dist_on, hbm_peak, "prefill_524k", 524288)
         extra["prefill_1m"] = leg_prefill(R, timer, args, dist_on, hbm_peak, "prefill_1m", 1 << 20)
         extra["build_2m"] = leg_build_2m(R, timer, args, dist_on, hbm_peak)
+        extra["decode_loop_1m"] = leg_decode_loop(R, timer, args, dist_on)
     clk = clocks.stop()
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

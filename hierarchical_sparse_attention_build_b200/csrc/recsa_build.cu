@@ -18,9 +18,13 @@ namespace {
 
 constexpr int kBuildThreads = 256;
 constexpr int kBuildWarps = kBuildThreads / 32;
+// Nodes per warp: 8 for a whole level; 1 for small launches (a prefill or decode step
+// extends one node per level and head), so their nodes run side by side, not in turn.
 constexpr int kNodesPerWarp = 8;
-constexpr int kNodesPerBlock = kBuildWarps * kNodesPerWarp;  // 64
-constexpr size_t kBuildSmem = (size_t)(kD * kD + kNodesPerBlock * kD) * sizeof(float);
+constexpr int kFewNodes = 1;
+__host__ __device__ constexpr size_t build_smem(int npw) {
+  return (size_t)(kD * kD + kBuildWarps * npw * kD) * sizeof(float);
+}
 
 struct BuildArgs {
   const uint16_t *src_k;  // level l-1 rows (token cache or node arena)
@@ -45,7 +49,9 @@ struct BuildArgs {
 // means in fp32, writes the value rows, then applies W to its own 8 key means (W^T
 // resident in shared memory, 8 nodes x 4 outputs per lane).  Warps share only W^T, so
 // they never wait for one another after it is loaded.
+template <int NPW>
 __global__ void __launch_bounds__(kBuildThreads, 2) build_level_kernel(const BuildArgs a) {
+  constexpr int kNodesPerBlock = kBuildWarps * NPW;
   extern __shared__ __align__(16) float smem_f[];
   float *Wt = smem_f;               // Wt[k][o] = W[o][k]
   float *Mean = smem_f + kD * kD;   // [64][128] key means
@@ -60,8 +66,8 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_level_kernel(const Bui
   const int64_t total = (int64_t)a.bh * a.nj;
   for (int64_t base = (int64_t)blockIdx.x * kNodesPerBlock; base < total;
        base += (int64_t)gridDim.x * kNodesPerBlock) {
-    for (int t = 0; t < kNodesPerWarp; ++t) {
-      const int nl = warp * kNodesPerWarp + t;
+    for (int t = 0; t < NPW; ++t) {
+      const int nl = warp * NPW + t;
       const int64_t id = base + nl;
       float2 ks2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // dims (0,1), (2,3) of the lane's 4
       float2 vs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
@@ -118,9 +124,9 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_level_kernel(const Bui
 
     // key = W @ mean for this warp's 8 nodes; lane owns outputs 4*lane .. 4*lane+3, as the
     // pairs (4l, 4l+1) and (4l+2, 4l+3) of packed fp32 FMAs (each output's terms in k order)
-    float2 acc2[kNodesPerWarp][2];
+    float2 acc2[NPW][2];
 #pragma unroll
-    for (int n = 0; n < kNodesPerWarp; ++n) acc2[n][0] = acc2[n][1] = make_float2(0.f, 0.f);
+    for (int n = 0; n < NPW; ++n) acc2[n][0] = acc2[n][1] = make_float2(0.f, 0.f);
     const float4 *Wt4 = reinterpret_cast<const float4 *>(Wt);
     const float4 *M4 = reinterpret_cast<const float4 *>(Mean);
 #pragma unroll 2
@@ -133,8 +139,8 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_level_kernel(const Bui
         w[t][1] = make_float2(wt.z, wt.w);
       }
 #pragma unroll
-      for (int n = 0; n < kNodesPerWarp; ++n) {
-        const float4 m = M4[(warp * kNodesPerWarp + n) * 32 + (k >> 2)];
+      for (int n = 0; n < NPW; ++n) {
+        const float4 m = M4[(warp * NPW + n) * 32 + (k >> 2)];
         const float mt[4] = {m.x, m.y, m.z, m.w};
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
@@ -144,17 +150,17 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_level_kernel(const Bui
         }
       }
     }
-    float acc[kNodesPerWarp][4];
+    float acc[NPW][4];
 #pragma unroll
-    for (int n = 0; n < kNodesPerWarp; ++n) {
+    for (int n = 0; n < NPW; ++n) {
       acc[n][0] = acc2[n][0].x;
       acc[n][1] = acc2[n][0].y;
       acc[n][2] = acc2[n][1].x;
       acc[n][3] = acc2[n][1].y;
     }
 #pragma unroll
-    for (int n = 0; n < kNodesPerWarp; ++n) {
-      const int64_t id = base + warp * kNodesPerWarp + n;
+    for (int n = 0; n < NPW; ++n) {
+      const int64_t id = base + warp * NPW + n;
       if (id < total) {
         const int64_t bhi = id / a.nj;
         const int64_t j = a.j0 + id % a.nj;
@@ -253,14 +259,24 @@ int launch_build_level(const TreeGeom &g, const recsa_tree &t, int level, int64_
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(build_level_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kBuildSmem);
+    cudaError_t e = cudaFuncSetAttribute(build_level_kernel<kNodesPerWarp>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)build_smem(kNodesPerWarp));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(build_level_kernel<kFewNodes>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)build_smem(kFewNodes));
     if (e != cudaSuccess) return (int)e;
     configured_device = dev;
   }
-  const int64_t blocks_needed = ceil_div((int64_t)a.bh * a.nj, kNodesPerBlock);
-  const int64_t grid = std::min<int64_t>(blocks_needed, (int64_t)sm_count() * 2);
-  build_level_kernel<<<(unsigned)grid, kBuildThreads, kBuildSmem, (cudaStream_t)stream>>>(a);
+  const int64_t nodes = (int64_t)a.bh * a.nj;
+  const int64_t full_grid = (int64_t)sm_count() * 2;
+  if (nodes <= full_grid * kBuildWarps * kFewNodes) {  // fits one pass of warps with a node each
+    const int64_t grid = ceil_div(nodes, kBuildWarps * kFewNodes);
+    build_level_kernel<kFewNodes><<<(unsigned)grid, kBuildThreads, build_smem(kFewNodes), (cudaStream_t)stream>>>(a);
+  } else {
+    const int64_t grid = std::min<int64_t>(ceil_div(nodes, kBuildWarps * kNodesPerWarp), full_grid);
+    build_level_kernel<kNodesPerWarp>
+        <<<(unsigned)grid, kBuildThreads, build_smem(kNodesPerWarp), (cudaStream_t)stream>>>(a);
+  }
   return (int)cudaGetLastError();
 }
 
