@@ -292,38 +292,50 @@ def leg_prefill(R, timer, args, dist_on, hbm_peak, name, length):
 
 
 def leg_decode_loop(R, timer, args, dist_on):
-    """Token-by-token decode at 1M (B = 4): every step appends one token to each sequence
-    (its K and V), extends the tree over it and attends that token's query, i.e.
-    recsa_prefill_chunk with a chunk of 1 -- the step a decode loop runs per token."""
+    """Token-by-token decode at 1M (B = 4).  A decode-loop step appends the step's token to
+    every sequence and updates the tree over it (recsa_append: the token slot and its
+    ancestor path, one launch), then decodes that token's query over all tokens so far
+    (recsa_decode).  Also timed: the same step as a causal chunk of one token
+    (recsa_prefill_chunk with C = 1).  Each step grows the cache by one token."""
     w = I.WORKLOADS["decode_1m"]
     warmup, steps = 4, 64 if not args.quick else 16
-    inp = I.decode_inputs(w, device="cuda", capacity=w.length + warmup + steps + 8)
+    per_leg = warmup + steps
+    inp = I.decode_inputs(w, device="cuda", capacity=w.length + 2 * per_leg + 8)
     p = R.params(num_kv_heads=w.kv_heads, num_q_heads=w.q_heads, branching=w.branching, top_k=w.top_k)
     tree, ws = make_tree(R, p, inp, w.length)
     g = torch.Generator(device="cuda").manual_seed(91)
     B, Hkv, Hq = w.batch, w.kv_heads, w.q_heads
     toks = [tuple(torch.randn(B, 1, h, 128, generator=g, device="cuda").to(torch.bfloat16) for h in (Hkv, Hkv, Hq))
-            for _ in range(warmup + steps + 1)]
+            for _ in range(2 * per_leg)]
     out = torch.empty(B, 1, Hq, 128, dtype=torch.bfloat16, device="cuda")
     nxt = [0]
 
-    def step():
+    def append_decode():
+        kn, vn, qn = toks[nxt[0]]
+        nxt[0] += 1
+        R.append(p, tree, kn, vn)
+        R.decode(p, tree, qn, out, ws)
+
+    def chunk_of_one():
         kn, vn, qn = toks[nxt[0]]
         nxt[0] += 1
         R.prefill_chunk(p, tree, kn, vn, qn, out, ws)
 
-    per, _ = timer.run(step, steps, warmup)
+    per, _ = timer.run(append_decode, steps, warmup)
     t = max_over_ranks(sum(per), dist_on) / steps
+    per, _ = timer.run(chunk_of_one, steps, warmup)
+    t_chunk = max_over_ranks(sum(per), dist_on) / steps
     R.check_device_errors(ws)
-    levels = tree.levels
     del tree, ws, inp
     torch.cuda.empty_cache()
     return {"workload": f"decode_loop_1m: B={B}, L={w.length} + 1 token per sequence per step, Hq={Hq}, "
                         f"Hkv={Hkv}, b={w.branching}, k={w.top_k}",
-            "tokens_per_s": B / t, "us_per_step": t * 1e6,
-            "launches_per_step": 2 + levels,
-            "note": "append + the tree extension (one node per level per head) + causal attend of the new "
-                    "token; each step grows the cache by one token"}
+            "tokens_per_s": B / t, "us_per_step": t * 1e6, "launches_per_step": 2,
+            "note": "recsa_append (token slot + ancestor path of every (sequence, KV head), one launch) + "
+                    "recsa_decode of the new token's query; L2 flushed before each step",
+            "causal_chunk_of_1": {"us_per_step": t_chunk * 1e6, "launches_per_step": 2,
+                                  "note": "recsa_prefill_chunk with C = 1: the same update, then the causal "
+                                          "attend (the partial node on the query's path always expanded)"}}
 
 
 def leg_build_2m(R, timer, args, dist_on, hbm_peak):

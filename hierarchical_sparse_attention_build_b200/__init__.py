@@ -95,6 +95,7 @@ def _load() -> ctypes.CDLL:
         "recsa_build_tree": [P, T, vp],
         "recsa_decode": [P, T, vp, i32, vp, i32, vp, sz, D, vp],
         "recsa_decode_host": [P, T, vp, i32, vp, i32, vp, vp, vp, sz, D, vp],
+        "recsa_append": [P, T, vp, vp, i32, vp],
         "recsa_prefill_chunk": [P, T, vp, vp, vp, i32, vp, i32, vp, sz, D, vp],
         "recsa_check_device_errors": [vp, vp],
         "recsa_decode_no_alloc": [P, T, vp, i32, vp, i32, vp],
@@ -238,6 +239,14 @@ def decode_host(p: Params, tree: RecsaTree, q_host: torch.Tensor, out_host: torc
     _check(_lib.recsa_decode_host(ctypes.byref(p), ctypes.byref(tree.c), _ptr(q_host), q_host.shape[1],
                                   _ptr(out_host), int(out_host.dtype == torch.float32), _ptr(q_dev), _ptr(out_dev),
                                   _ptr(ws.buf), ws.nbytes, None, _stream(stream)))
+
+
+def append(p: Params, tree: RecsaTree, k_new: torch.Tensor, v_new: torch.Tensor, stream=None) -> None:
+    """recsa_append: append [B][C][Hkv][128] K/V to every sequence and rebuild the nodes over them."""
+    for t in (k_new, v_new):
+        assert t.dtype == torch.bfloat16 and t.is_contiguous()
+    _check(_lib.recsa_append(ctypes.byref(p), ctypes.byref(tree.c), _ptr(k_new), _ptr(v_new), k_new.shape[1],
+                             _stream(stream)))
 
 
 def prefill_chunk(p: Params, tree: RecsaTree, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor,

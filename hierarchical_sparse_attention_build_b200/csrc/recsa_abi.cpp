@@ -175,6 +175,34 @@ recsa_status build_range(const TreeGeom &g, const recsa_tree &t, int64_t length,
   return RECSA_OK;
 }
 
+// Appends `chunk` tokens at L and rebuilds every node whose span meets them.  When the chunk
+// is short and each level has at most kPathNodes such nodes per (sequence, head) (a decode
+// step's token, a short prefill chunk), one launch appends and walks the ancestor path, a
+// warp per (sequence, head); otherwise the tokens are copied and each level is rebuilt by
+// its own launch, wide over the level's nodes.
+constexpr int64_t kPathNodes = 4;
+constexpr int kPathTokens = 64;
+recsa_status extend_tree(const TreeGeom &g, const recsa_tree &t, const void *k_new, const void *v_new, int64_t L,
+                         int chunk, void *stream) {
+  const int64_t L2 = L + chunk;
+  const int T_new = levels_for(L2, g.b);
+  const int T_old = levels_for(L, g.b);
+  int64_t j0[kMaxLevels + 1] = {0}, j1[kMaxLevels + 1] = {0};
+  int64_t most = 0;
+  for (int l = 1; l <= T_new; ++l) {
+    j0[l] = l <= T_old ? L / g.span[l] : 0;
+    j1[l] = ceil_div(L2, g.span[l]);
+    most = std::max(most, j1[l] - j0[l]);
+  }
+  if (chunk <= kPathTokens && most <= kPathNodes) {
+    const int rc = launch_extend(g, t, k_new, v_new, L, chunk, T_new, j0, j1, stream);
+    return rc != 0 ? cuda_fail(rc, "append and path update") : RECSA_OK;
+  }
+  const int rc = launch_append(g, t, k_new, v_new, L, chunk, stream);
+  if (rc != 0) return cuda_fail(rc, "append");
+  return build_range(g, t, L2, L, true, stream);
+}
+
 // Every check of a decode call and the launch it becomes (nothing is queued here).
 recsa_status decode_launch(const recsa_params *params, const recsa_tree *tree, const void *q, int32_t num_queries,
                            void *out, int32_t out_is_fp32, void *ws, size_t ws_bytes, const recsa_debug *debug,
@@ -335,6 +363,27 @@ RECSA_API recsa_status recsa_decode_host(const recsa_params *params, const recsa
   return RECSA_OK;
 }
 
+RECSA_API recsa_status recsa_append(const recsa_params *params, recsa_tree *tree, const void *k_new,
+                                    const void *v_new, int32_t count, recsa_stream_t stream) {
+  recsa_status s = check_params(params);
+  if (s != RECSA_OK) return s;
+  TreeGeom g;
+  s = check_tree(params, tree, &g);
+  if (s != RECSA_OK) return s;
+  if (count < 1) return fail(RECSA_ERR_INVALID_ARGUMENT, "count %d < 1", count);
+  if (!k_new || !v_new) return fail(RECSA_ERR_INVALID_ARGUMENT, "k_new or v_new is NULL");
+  if (!aligned16(k_new) || !aligned16(v_new))
+    return fail(RECSA_ERR_INVALID_ARGUMENT, "k_new or v_new is not 16-byte aligned");
+  const int64_t L = tree->length;
+  if (L + count > tree->capacity)
+    return fail(RECSA_ERR_CAPACITY, "length %lld + count %d > capacity %lld", (long long)L, count,
+                (long long)tree->capacity);
+  s = extend_tree(g, *tree, k_new, v_new, L, count, stream);
+  if (s != RECSA_OK) return s;
+  tree->length = L + count;
+  return RECSA_OK;
+}
+
 RECSA_API recsa_status recsa_prefill_chunk(const recsa_params *params, recsa_tree *tree, const void *k_new,
                                            const void *v_new, const void *q, int32_t chunk, void *out,
                                            int32_t out_is_fp32, void *ws, size_t ws_bytes, const recsa_debug *debug,
@@ -363,9 +412,7 @@ RECSA_API recsa_status recsa_prefill_chunk(const recsa_params *params, recsa_tre
   const int64_t tiles = (int64_t)tree->batch * params->num_kv_heads * chunk;
   if (tiles > 0x7fffffff / 4) return fail(RECSA_ERR_UNSUPPORTED, "%lld tiles", (long long)tiles);
 
-  int rc = launch_append(g, *tree, k_new, v_new, L, chunk, stream);
-  if (rc != 0) return cuda_fail(rc, "append");
-  s = build_range(g, *tree, L2, L, true, stream);
+  s = extend_tree(g, *tree, k_new, v_new, L, chunk, stream);
   if (s != RECSA_OK) return s;
   AttendLaunch l;
   l.geom = g;
@@ -385,7 +432,7 @@ RECSA_API recsa_status recsa_prefill_chunk(const recsa_params *params, recsa_tre
   l.cluster_size = debug ? debug->cluster_size : 0;
   l.kernel = debug ? debug->kernel : 0;
   l.debug = debug;
-  rc = launch_attend(l, stream);
+  const int rc = launch_attend(l, stream);
   if (rc != 0) return cuda_fail(rc, "prefill attend");
   tree->length = L2;
   return RECSA_OK;

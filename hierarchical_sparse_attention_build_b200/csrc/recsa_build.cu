@@ -1,4 +1,5 @@
-// Tree build (one level per launch), chunk append and RoPE table kernels.
+// Tree build (one level per launch), append with path update (all levels in one launch),
+// chunk append and RoPE table kernels.
 //
 // Recursive Sparse Attention, abstract: every node summarises its subtree with one
 // key, made by a per-layer pooler shared by all levels, and one mean-pooled value.
@@ -44,23 +45,142 @@ struct BuildArgs {
   const float *pooler;    // [128][128] row-major W
 };
 
-// One CTA handles blocks of 64 nodes: each warp streams the children of 8 nodes
-// (lane = 4 consecutive dims, one 256-byte row per warp load), forms the child
-// means in fp32, writes the value rows, then applies W to its own 8 key means (W^T
-// resident in shared memory, 8 nodes x 4 outputs per lane).  Warps share only W^T, so
-// they never wait for one another after it is loaded.
+// Wt[k][o] = W[o][k] into shared memory.  A thread moves 16-byte pieces of W; the 32 lanes of
+// a warp take 32 consecutive rows o at the same column, so each shared-memory store fills 32
+// banks, and a thread's pieces are all loaded before any is stored.
+template <int NT>
+__device__ __forceinline__ void load_wt(const float *__restrict__ W, float *Wt, int tid) {
+  constexpr int kPieces = kD * kD / 4 / NT;
+  static_assert(kD * kD / 4 % NT == 0, "threads must divide the pooler's 16-byte pieces");
+  float4 w[kPieces];
+#pragma unroll
+  for (int i = 0; i < kPieces; ++i) {
+    const int e = tid + i * NT;  // piece e: row o = e % 128, columns 4 * (e / 128) .. +3
+    w[i] = __ldg(reinterpret_cast<const float4 *>(W) + (e & (kD - 1)) * (kD / 4) + (e >> 7));
+  }
+#pragma unroll
+  for (int i = 0; i < kPieces; ++i) {
+    const int e = tid + i * NT;
+    const int o = e & (kD - 1), k = (e >> 7) * 4;
+    Wt[(k + 0) * kD + o] = w[i].x;
+    Wt[(k + 1) * kD + o] = w[i].y;
+    Wt[(k + 2) * kD + o] = w[i].z;
+    Wt[(k + 3) * kD + o] = w[i].w;
+  }
+}
+
+// One child row piece (the lane's 4 dims): through the read-only path for a level written by
+// an earlier launch, an ordinary load for one this kernel may have written.
+template <bool kReadOnly>
+__device__ __forceinline__ uint2 ld_child(const uint16_t *p) {
+  if constexpr (kReadOnly)
+    return __ldg(reinterpret_cast<const uint2 *>(p));
+  else
+    return *reinterpret_cast<const uint2 *>(p);
+}
+
+// The lane's 4 dims of node means over children [c0, c1) of level l-1 (kb, vb point at the
+// lane's dims of the (sequence, head) block's first row).  Key: plain mean of the children's
+// stored keys.  Value: token-count-weighted mean; every child but the level's last covers
+// span_prev tokens, so the children are summed with weight 1 and the last child, if it covers
+// fewer tokens, then gets its share f = tokens / span_prev.
+template <bool kReadOnly>
+__device__ __forceinline__ void node_means(const uint16_t *kb, const uint16_t *vb, int64_t c0, int64_t c1,
+                                           int64_t n_prev, int64_t length, int64_t span_prev, float ks[4],
+                                           float vs[4]) {
+  float2 ks2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // dims (0,1), (2,3) of the lane's 4
+  float2 vs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll 16  // a whole node's children (b = 16) in flight at once
+  for (int64_t c = c0; c < c1; ++c) {
+    const uint2 ku = ld_child<kReadOnly>(kb + c * kD);
+    const uint2 vu = ld_child<kReadOnly>(vb + c * kD);
+    ks2[0] = __fadd2_rn(ks2[0], make_float2(bf16_lo(ku.x), bf16_hi(ku.x)));
+    ks2[1] = __fadd2_rn(ks2[1], make_float2(bf16_lo(ku.y), bf16_hi(ku.y)));
+    vs2[0] = __fadd2_rn(vs2[0], make_float2(bf16_lo(vu.x), bf16_hi(vu.x)));
+    vs2[1] = __fadd2_rn(vs2[1], make_float2(bf16_lo(vu.y), bf16_hi(vu.y)));
+  }
+  ks[0] = ks2[0].x, ks[1] = ks2[0].y, ks[2] = ks2[1].x, ks[3] = ks2[1].y;
+  vs[0] = vs2[0].x, vs[1] = vs2[0].y, vs[2] = vs2[1].x, vs[3] = vs2[1].y;
+  const float nch = (float)(c1 - c0);
+  float wsum = nch;
+  if (c1 == n_prev && c1 > c0) {
+    const int64_t last_tokens = length - (c1 - 1) * span_prev;
+    if (last_tokens < span_prev) {
+      const float f1 = (float)last_tokens / (float)span_prev - 1.f;
+      const uint2 vu = ld_child<kReadOnly>(vb + (c1 - 1) * kD);
+      vs[0] = __fmaf_rn(f1, bf16_lo(vu.x), vs[0]);
+      vs[1] = __fmaf_rn(f1, bf16_hi(vu.x), vs[1]);
+      vs[2] = __fmaf_rn(f1, bf16_lo(vu.y), vs[2]);
+      vs[3] = __fmaf_rn(f1, bf16_hi(vu.y), vs[3]);
+      wsum += f1;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    ks[i] = ks[i] / nch;
+    vs[i] = vs[i] / wsum;
+  }
+}
+
+// key = W @ mean for NPW nodes whose key means are rows [NPW][128] in shared memory; lane
+// owns outputs 4*lane .. 4*lane+3, as the pairs (4l, 4l+1) and (4l+2, 4l+3) of packed fp32
+// FMAs (each output's terms in k order).
+template <int NPW>
+__device__ __forceinline__ void apply_w(const float *Wt, const float *mean_rows, int lane, float acc[NPW][4]) {
+  float2 acc2[NPW][2];
+#pragma unroll
+  for (int n = 0; n < NPW; ++n) acc2[n][0] = acc2[n][1] = make_float2(0.f, 0.f);
+  const float4 *Wt4 = reinterpret_cast<const float4 *>(Wt);
+  const float4 *M4 = reinterpret_cast<const float4 *>(mean_rows);
+#pragma unroll 2
+  for (int k = 0; k < kD; k += 4) {
+    float2 w[4][2];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const float4 wt = Wt4[(k + t) * 32 + lane];
+      w[t][0] = make_float2(wt.x, wt.y);
+      w[t][1] = make_float2(wt.z, wt.w);
+    }
+#pragma unroll
+    for (int n = 0; n < NPW; ++n) {
+      const float4 m = M4[n * 32 + (k >> 2)];
+      const float mt[4] = {m.x, m.y, m.z, m.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float2 mm = make_float2(mt[t], mt[t]);
+        acc2[n][0] = __ffma2_rn(mm, w[t][0], acc2[n][0]);
+        acc2[n][1] = __ffma2_rn(mm, w[t][1], acc2[n][1]);
+      }
+    }
+  }
+#pragma unroll
+  for (int n = 0; n < NPW; ++n) {
+    acc[n][0] = acc2[n][0].x;
+    acc[n][1] = acc2[n][0].y;
+    acc[n][2] = acc2[n][1].x;
+    acc[n][3] = acc2[n][1].y;
+  }
+}
+
+__device__ __forceinline__ void store_row4(uint16_t *p, const float x[4]) {
+  uint2 o;
+  o.x = pack_bf16x2(x[0], x[1]);
+  o.y = pack_bf16x2(x[2], x[3]);
+  *reinterpret_cast<uint2 *>(p) = o;
+}
+
+// One CTA handles blocks of 8 * NPW nodes: each warp streams the children of NPW nodes
+// (lane = 4 consecutive dims, one 256-byte row per warp load), forms the child means in
+// fp32, writes the value rows, then applies W to its own key means (W^T resident in shared
+// memory).  Warps share only W^T, so they never wait for one another after it is loaded.
 template <int NPW>
 __global__ void __launch_bounds__(kBuildThreads, 2) build_level_kernel(const BuildArgs a) {
   constexpr int kNodesPerBlock = kBuildWarps * NPW;
   extern __shared__ __align__(16) float smem_f[];
   float *Wt = smem_f;               // Wt[k][o] = W[o][k]
-  float *Mean = smem_f + kD * kD;   // [64][128] key means
+  float *Mean = smem_f + kD * kD;   // [8 * NPW][128] key means
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-
-  for (int e = tid; e < kD * kD; e += kBuildThreads) {
-    const int o = e >> 7, k = e & 127;
-    Wt[k * kD + o] = a.pooler[e];
-  }
+  load_wt<kBuildThreads>(a.pooler, Wt, tid);
   __syncthreads();
 
   const int64_t total = (int64_t)a.bh * a.nj;
@@ -69,8 +189,6 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_level_kernel(const Bui
     for (int t = 0; t < NPW; ++t) {
       const int nl = warp * NPW + t;
       const int64_t id = base + nl;
-      float2 ks2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // dims (0,1), (2,3) of the lane's 4
-      float2 vs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       float ks[4] = {0.f, 0.f, 0.f, 0.f}, vs[4] = {0.f, 0.f, 0.f, 0.f};
       if (id < total) {
         const int64_t bhi = id / a.nj;
@@ -79,98 +197,177 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_level_kernel(const Bui
         const int64_t c1 = min(c0 + (int64_t)a.b, a.n_prev);
         const uint16_t *kb = a.src_k + (a.src_row_off + bhi * a.src_slots) * kD + lane * 4;
         const uint16_t *vb = a.src_v + (a.src_row_off + bhi * a.src_slots) * kD + lane * 4;
-        // Every child but the level's last covers span_prev tokens, so the value mean
-        // sums the children with weight 1 and then gives the last child, if it covers
-        // fewer tokens, its share f = tokens / span_prev.
-#pragma unroll 16  // a whole node's children (b = 16) in flight at once
-        for (int64_t c = c0; c < c1; ++c) {
-          const uint2 ku = __ldg(reinterpret_cast<const uint2 *>(kb + c * kD));
-          const uint2 vu = __ldg(reinterpret_cast<const uint2 *>(vb + c * kD));
-          ks2[0] = __fadd2_rn(ks2[0], make_float2(bf16_lo(ku.x), bf16_hi(ku.x)));
-          ks2[1] = __fadd2_rn(ks2[1], make_float2(bf16_lo(ku.y), bf16_hi(ku.y)));
-          vs2[0] = __fadd2_rn(vs2[0], make_float2(bf16_lo(vu.x), bf16_hi(vu.x)));
-          vs2[1] = __fadd2_rn(vs2[1], make_float2(bf16_lo(vu.y), bf16_hi(vu.y)));
-        }
-        ks[0] = ks2[0].x, ks[1] = ks2[0].y, ks[2] = ks2[1].x, ks[3] = ks2[1].y;
-        vs[0] = vs2[0].x, vs[1] = vs2[0].y, vs[2] = vs2[1].x, vs[3] = vs2[1].y;
-        const float nch = (float)(c1 - c0);
-        float wsum = nch;
-        if (c1 == a.n_prev && c1 > c0) {
-          const int64_t last_tokens = a.length - (c1 - 1) * a.span_prev;
-          if (last_tokens < a.span_prev) {
-            const float f1 = (float)last_tokens / (float)a.span_prev - 1.f;
-            const uint2 vu = __ldg(reinterpret_cast<const uint2 *>(vb + (c1 - 1) * kD));
-            vs[0] += f1 * bf16_lo(vu.x);
-            vs[1] += f1 * bf16_hi(vu.x);
-            vs[2] += f1 * bf16_lo(vu.y);
-            vs[3] += f1 * bf16_hi(vu.y);
-            wsum += f1;
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          ks[i] = ks[i] / nch;
-          vs[i] = vs[i] / wsum;
-        }
-        uint2 vo;
-        vo.x = pack_bf16x2(vs[0], vs[1]);
-        vo.y = pack_bf16x2(vs[2], vs[3]);
-        *reinterpret_cast<uint2 *>(a.dst_v + (a.dst_row_off + bhi * a.dst_slots + j) * kD + lane * 4) = vo;
+        node_means<true>(kb, vb, c0, c1, a.n_prev, a.length, a.span_prev, ks, vs);
+        store_row4(a.dst_v + (a.dst_row_off + bhi * a.dst_slots + j) * kD + lane * 4, vs);
       }
       *reinterpret_cast<float4 *>(Mean + nl * kD + lane * 4) = make_float4(ks[0], ks[1], ks[2], ks[3]);
     }
-    __syncwarp();  // a warp applies W to its own 8 nodes only: warps run out of step, so some
+    __syncwarp();  // a warp applies W to its own nodes only: warps run out of step, so some
                    // stream children while others compute
-
-    // key = W @ mean for this warp's 8 nodes; lane owns outputs 4*lane .. 4*lane+3, as the
-    // pairs (4l, 4l+1) and (4l+2, 4l+3) of packed fp32 FMAs (each output's terms in k order)
-    float2 acc2[NPW][2];
-#pragma unroll
-    for (int n = 0; n < NPW; ++n) acc2[n][0] = acc2[n][1] = make_float2(0.f, 0.f);
-    const float4 *Wt4 = reinterpret_cast<const float4 *>(Wt);
-    const float4 *M4 = reinterpret_cast<const float4 *>(Mean);
-#pragma unroll 2
-    for (int k = 0; k < kD; k += 4) {
-      float2 w[4][2];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const float4 wt = Wt4[(k + t) * 32 + lane];
-        w[t][0] = make_float2(wt.x, wt.y);
-        w[t][1] = make_float2(wt.z, wt.w);
-      }
-#pragma unroll
-      for (int n = 0; n < NPW; ++n) {
-        const float4 m = M4[(warp * NPW + n) * 32 + (k >> 2)];
-        const float mt[4] = {m.x, m.y, m.z, m.w};
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const float2 mm = make_float2(mt[t], mt[t]);
-          acc2[n][0] = __ffma2_rn(mm, w[t][0], acc2[n][0]);
-          acc2[n][1] = __ffma2_rn(mm, w[t][1], acc2[n][1]);
-        }
-      }
-    }
     float acc[NPW][4];
-#pragma unroll
-    for (int n = 0; n < NPW; ++n) {
-      acc[n][0] = acc2[n][0].x;
-      acc[n][1] = acc2[n][0].y;
-      acc[n][2] = acc2[n][1].x;
-      acc[n][3] = acc2[n][1].y;
-    }
+    apply_w<NPW>(Wt, Mean + warp * NPW * kD, lane, acc);
 #pragma unroll
     for (int n = 0; n < NPW; ++n) {
       const int64_t id = base + warp * NPW + n;
       if (id < total) {
         const int64_t bhi = id / a.nj;
         const int64_t j = a.j0 + id % a.nj;
-        uint2 ko;
-        ko.x = pack_bf16x2(acc[n][0], acc[n][1]);
-        ko.y = pack_bf16x2(acc[n][2], acc[n][3]);
-        *reinterpret_cast<uint2 *>(a.dst_k + (a.dst_row_off + bhi * a.dst_slots + j) * kD + lane * 4) = ko;
+        store_row4(a.dst_k + (a.dst_row_off + bhi * a.dst_slots + j) * kD + lane * 4, acc[n]);
       }
     }
     __syncwarp();  // this warp's Mean rows are rewritten next
+  }
+}
+
+// Append and path update in one launch: one CTA per (sequence, KV head).  The CTA copies
+// its chunk of new tokens into the token cache, then walks up the levels and rebuilds, at
+// each level l, the nodes [j0[l], j1[l]) whose spans meet the new tokens (the nodes above
+// them are those nodes' ancestors).  A thread owns one dimension of the key (threads
+// 0..127) or of the value (128..255): it sums that dimension over the node's children and
+// forms its mean.  The key output o = W[o] . mean is one fp32 FMA chain over k = 0..127: the
+// key thread of dimension o runs k < 64 and the value thread of the same o continues with
+// k >= 64, each with its half of W row o in registers.  Per element these are the level
+// build's operations in the level build's order, so the extended tree equals a full build
+// bit for bit.  Rows written at level l are read at level l+1 by other threads of the same
+// CTA after a __syncthreads; no two CTAs touch the same rows.
+struct ExtendArgs {
+  const uint4 *k_new, *v_new;   // [B][C][Hkv][128] bf16, as 16-byte pieces
+  uint16_t *k_tok, *v_tok;      // [B][Hkv][capacity][128]
+  uint16_t *k_node, *v_node;    // node arena
+  const float *pooler;
+  int64_t capacity;
+  int64_t at;                   // first new slot (the length before the append)
+  int64_t length;               // length after it
+  int32_t chunk, hkv, b, levels;  // levels = T(length)
+  int64_t row_off[kMaxLevels + 1];
+  int64_t slots[kMaxLevels + 1];
+  int64_t span[kMaxLevels + 1];
+  int64_t j0[kMaxLevels + 1], j1[kMaxLevels + 1];  // nodes rebuilt at level l
+};
+constexpr int kExtendThreads = 2 * kD;  // one thread per key dimension and per value dimension
+constexpr int kHalfK = kD / 2;          // W columns held by each thread of a dimension
+// W^T staged as Wt[k][o ^ (k / 4 % 32)]: the coalesced row loads (a warp reads one W row)
+// and the per-thread row reads both hit 32 distinct banks.
+constexpr size_t kExtendSmem = (size_t)(kD * kD + 2 * kD) * sizeof(float);
+
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+__global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendArgs a) {
+  extern __shared__ __align__(16) float smem_f[];
+  float *Wt = smem_f;               // swizzled W^T (staging only)
+  float *mean = smem_f + kD * kD;   // the node's key mean
+  float *part = mean + kD;          // key outputs after k < 64
+  const int tid = threadIdx.x;
+  const int64_t bhi = blockIdx.x;   // (sequence, head)
+  const int d = tid & (kD - 1);
+  const bool is_v = tid >= kD;
+
+  // W in flight (a warp reads one 512-byte row) while the tokens are appended and the first
+  // children load
+  constexpr int kPieces = kD * kD / 4 / kExtendThreads;
+  float4 w[kPieces];
+#pragma unroll
+  for (int i = 0; i < kPieces; ++i) w[i] = __ldg(reinterpret_cast<const float4 *>(a.pooler) + tid + i * kExtendThreads);
+  {
+    const int64_t s = bhi / a.hkv, h = bhi % a.hkv;
+    uint4 *kt = reinterpret_cast<uint4 *>(a.k_tok + (bhi * a.capacity + a.at) * kD);
+    uint4 *vt = reinterpret_cast<uint4 *>(a.v_tok + (bhi * a.capacity + a.at) * kD);
+    for (int e = tid; e < a.chunk * 16; e += kExtendThreads) {  // 16 pieces a row
+      const int64_t src = ((s * a.chunk + (e >> 4)) * a.hkv + h) * 16 + (e & 15);
+      kt[e] = __ldg(a.k_new + src);
+      vt[e] = __ldg(a.v_new + src);
+    }
+  }
+  // every child row the walk reads above level 1, into L2 ahead of the dependent levels
+  // (K and V, two 128-byte lines each)
+  for (int l = 2; l <= a.levels; ++l) {
+    const int64_t n_prev = (a.length + a.span[l - 1] - 1) / a.span[l - 1];
+    const int64_t c0 = a.j0[l] * a.b, c1 = min(a.j1[l] * a.b, n_prev);
+    const int64_t base = (a.row_off[l - 1] + bhi * a.slots[l - 1]) * kD;
+    for (int64_t e = tid; e < (c1 - c0) * 4; e += kExtendThreads)
+      prefetch_l2(((e & 2) ? a.v_node : a.k_node) + base + (c0 + (e >> 2)) * kD + (e & 1) * (kD / 2));
+  }
+  __syncthreads();  // the appended rows are read below by other threads
+
+  float wr[kHalfK];  // W[d][64 * is_v + i]
+  bool w_ready = false;
+  const int kbase = is_v ? kHalfK : 0;
+  for (int l = 1; l <= a.levels; ++l) {
+    const int64_t span_prev = a.span[l - 1];
+    const int64_t n_prev = (a.length + span_prev - 1) / span_prev;
+    const uint16_t *src = l == 1 ? (is_v ? a.v_tok : a.k_tok) + bhi * a.capacity * kD
+                                 : (is_v ? a.v_node : a.k_node) + (a.row_off[l - 1] + bhi * a.slots[l - 1]) * kD;
+    uint16_t *dk = a.k_node + (a.row_off[l] + bhi * a.slots[l]) * kD;
+    uint16_t *dv = a.v_node + (a.row_off[l] + bhi * a.slots[l]) * kD;
+    for (int64_t j = a.j0[l]; j < a.j1[l]; ++j) {
+      const int64_t c0 = j * a.b, c1 = min(c0 + (int64_t)a.b, n_prev);
+      float sum = 0.f;
+#pragma unroll 16
+      for (int64_t c = c0; c < c1; ++c) sum += bf16_lo(src[c * kD + d]);
+      const float nch = (float)(c1 - c0);
+      if (is_v) {  // token-weighted: the level's last child gets its share tokens / span_prev
+        float wsum = nch;
+        if (c1 == n_prev && c1 > c0) {
+          const int64_t last_tokens = a.length - (c1 - 1) * span_prev;
+          if (last_tokens < span_prev) {
+            const float f1 = (float)last_tokens / (float)span_prev - 1.f;
+            sum = __fmaf_rn(f1, bf16_lo(src[(c1 - 1) * kD + d]), sum);
+            wsum += f1;
+          }
+        }
+        dv[j * kD + d] = (uint16_t)f32_to_bf16_bits(sum / wsum);
+      } else {
+        mean[d] = sum / nch;
+      }
+      if (!w_ready) {  // first node: W^T through shared memory into each thread's registers
+#pragma unroll
+        for (int i = 0; i < kPieces; ++i) {
+          const int e = tid + i * kExtendThreads;
+          const int o = e >> 5, q = e & 31;  // W[o][4q .. 4q+3]
+          Wt[(4 * q + 0) * kD + (o ^ q)] = w[i].x;
+          Wt[(4 * q + 1) * kD + (o ^ q)] = w[i].y;
+          Wt[(4 * q + 2) * kD + (o ^ q)] = w[i].z;
+          Wt[(4 * q + 3) * kD + (o ^ q)] = w[i].w;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < kHalfK; ++i) {
+          const int k = kbase + i;
+          wr[i] = Wt[k * kD + (d ^ ((k >> 2) & 31))];
+        }
+        w_ready = true;
+      }
+      __syncthreads();  // the key mean in place
+      const float4 *m4 = reinterpret_cast<const float4 *>(mean + kbase);
+      float acc = 0.f;
+      if (!is_v) {
+#pragma unroll
+        for (int i = 0; i < kHalfK / 4; ++i) {
+          const float4 m = m4[i];
+          acc = __fmaf_rn(m.x, wr[4 * i + 0], acc);
+          acc = __fmaf_rn(m.y, wr[4 * i + 1], acc);
+          acc = __fmaf_rn(m.z, wr[4 * i + 2], acc);
+          acc = __fmaf_rn(m.w, wr[4 * i + 3], acc);
+        }
+        part[d] = acc;
+      }
+      __syncthreads();  // the first half of every key output in place
+      if (is_v) {
+        acc = part[d];
+#pragma unroll
+        for (int i = 0; i < kHalfK / 4; ++i) {
+          const float4 m = m4[i];
+          acc = __fmaf_rn(m.x, wr[4 * i + 0], acc);
+          acc = __fmaf_rn(m.y, wr[4 * i + 1], acc);
+          acc = __fmaf_rn(m.z, wr[4 * i + 2], acc);
+          acc = __fmaf_rn(m.w, wr[4 * i + 3], acc);
+        }
+        dk[j * kD + d] = (uint16_t)f32_to_bf16_bits(acc);
+      }
+      __syncthreads();  // mean and part are rewritten next, and the next level reads these rows
+    }
   }
 }
 
@@ -222,6 +419,25 @@ int sm_count() {
   return n;
 }
 
+// Dynamic shared memory above 48 KB is opted into once per device and host thread.
+int configure_smem() {
+  static thread_local int configured_device = -1;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return (int)e;
+  if (configured_device == dev) return 0;
+  e = cudaFuncSetAttribute(build_level_kernel<kNodesPerWarp>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)build_smem(kNodesPerWarp));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(build_level_kernel<kFewNodes>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)build_smem(kFewNodes));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(extend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kExtendSmem);
+  if (e != cudaSuccess) return (int)e;
+  configured_device = dev;
+  return 0;
+}
+
 }  // namespace
 
 int launch_rope_table(void *ws, int rows, double base, void *stream) {
@@ -255,18 +471,8 @@ int launch_build_level(const TreeGeom &g, const recsa_tree &t, int level, int64_
   a.b = g.b;
   a.bh = g.batch * g.hkv;
   a.pooler = t.pooler;
-  static thread_local int configured_device = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(build_level_kernel<kNodesPerWarp>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)build_smem(kNodesPerWarp));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(build_level_kernel<kFewNodes>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)build_smem(kFewNodes));
-    if (e != cudaSuccess) return (int)e;
-    configured_device = dev;
-  }
+  const int rc = configure_smem();
+  if (rc != 0) return rc;
   const int64_t nodes = (int64_t)a.bh * a.nj;
   const int64_t full_grid = (int64_t)sm_count() * 2;
   if (nodes <= full_grid * kBuildWarps * kFewNodes) {  // fits one pass of warps with a node each
@@ -277,6 +483,37 @@ int launch_build_level(const TreeGeom &g, const recsa_tree &t, int level, int64_
     build_level_kernel<kNodesPerWarp>
         <<<(unsigned)grid, kBuildThreads, build_smem(kNodesPerWarp), (cudaStream_t)stream>>>(a);
   }
+  return (int)cudaGetLastError();
+}
+
+int launch_extend(const TreeGeom &g, const recsa_tree &t, const void *k_new, const void *v_new, int64_t at,
+                  int chunk, int levels, const int64_t *j0, const int64_t *j1, void *stream) {
+  ExtendArgs a;
+  a.k_new = reinterpret_cast<const uint4 *>(k_new);
+  a.v_new = reinterpret_cast<const uint4 *>(v_new);
+  a.k_tok = reinterpret_cast<uint16_t *>(t.k_tok);
+  a.v_tok = reinterpret_cast<uint16_t *>(t.v_tok);
+  a.k_node = reinterpret_cast<uint16_t *>(t.k_node);
+  a.v_node = reinterpret_cast<uint16_t *>(t.v_node);
+  a.pooler = t.pooler;
+  a.capacity = g.capacity;
+  a.at = at;
+  a.length = at + chunk;
+  a.chunk = chunk;
+  a.hkv = g.hkv;
+  a.b = g.b;
+  a.levels = levels;
+  for (int l = 0; l <= kMaxLevels; ++l) {
+    a.row_off[l] = g.row_off[l];
+    a.slots[l] = g.slots[l];
+    a.span[l] = g.span[l];
+    a.j0[l] = l <= levels ? j0[l] : 0;
+    a.j1[l] = l <= levels ? j1[l] : 0;
+  }
+  const int rc = configure_smem();
+  if (rc != 0) return rc;
+  const int64_t grid = (int64_t)g.batch * g.hkv;
+  extend_kernel<<<(unsigned)grid, kExtendThreads, kExtendSmem, (cudaStream_t)stream>>>(a);
   return (int)cudaGetLastError();
 }
 

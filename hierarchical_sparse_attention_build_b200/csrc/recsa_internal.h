@@ -55,6 +55,10 @@ int launch_build_level(const TreeGeom &g, const recsa_tree &t, int level, int64_
                        void *stream);
 int launch_append(const TreeGeom &g, const recsa_tree &t, const void *k_new, const void *v_new, int64_t at,
                   int chunk, void *stream);
+// Append `chunk` tokens at slot `at` and rebuild nodes [j0[l], j1[l]) of levels 1..levels in
+// one launch (one warp per (sequence, head) walks up the levels).
+int launch_extend(const TreeGeom &g, const recsa_tree &t, const void *k_new, const void *v_new, int64_t at,
+                  int chunk, int levels, const int64_t *j0, const int64_t *j1, void *stream);
 
 struct AttendLaunch {
   TreeGeom geom;

@@ -190,6 +190,21 @@ RECSA_API recsa_status recsa_decode_host(const recsa_params *params, const recsa
                                          void *out_dev, void *ws, size_t ws_bytes, const recsa_debug *debug,
                                          recsa_stream_t stream);
 
+/* Append `count` tokens to every sequence and update the tree over them (abstract:
+ * trees over the KV cache; the incremental update is not specified there): k_new /
+ * v_new go to token slots L .. L+count-1 (L = tree->length), and every node whose span
+ * meets those slots is rebuilt from its children -- the new tokens' ancestors, O(T)
+ * nodes per (sequence, head) for one token -- plus any level that becomes new.  The
+ * result equals recsa_build_tree over L + count tokens.  This is the cache update of a
+ * decode loop: append the step's token, then recsa_decode its query at the new length.
+ * On success tree->length becomes L + count (host-side update; the device work is
+ * still queued).
+ *   k_new, v_new: bf16 [batch][count][Hkv][128] (device, 16-byte aligned).
+ * Needs count >= 1 and L + count <= capacity (else RECSA_ERR_CAPACITY); nothing is
+ * queued when a check fails. */
+RECSA_API recsa_status recsa_append(const recsa_params *params, recsa_tree *tree, const void *k_new,
+                                    const void *v_new, int32_t count, recsa_stream_t stream);
+
 /* Causal prefill of a chunk of `chunk` tokens at positions L .. L+chunk-1
  * (L = tree->length): appends k_new / v_new to the token caches, rebuilds the tree
  * nodes those tokens touch (and any level that becomes new), then attends query i

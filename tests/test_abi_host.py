@@ -29,7 +29,7 @@ def test_library_exports_every_declared_symbol():
     names = declared_functions()
     assert set(names) == {"recsa_tree_layout", "recsa_workspace_size", "recsa_workspace_init", "recsa_build_tree",
                           "recsa_decode", "recsa_prefill_chunk", "recsa_check_device_errors", "recsa_status_string",
-                          "recsa_last_error", "recsa_decode_no_alloc", "recsa_decode_host"}, names
+                          "recsa_last_error", "recsa_decode_no_alloc", "recsa_decode_host", "recsa_append"}, names
     for n in names:
         assert hasattr(lib, n), n
         assert ctypes.cast(getattr(lib, n), ctypes.c_void_p).value
@@ -161,6 +161,21 @@ def test_prefill_capacity_and_arguments_rejected():
     assert call(t, k=0) == INVALID
     assert call(t, v=FAKE + 2) == INVALID
     assert call(t, ws=10) == WS_SMALL
+    assert t.length == 4000  # unchanged on failure
+
+
+def test_append_capacity_and_arguments_rejected():
+    p = _p()
+    t = _tree(length=4000)
+    call = lambda t, count=64, **kw: lib.recsa_append(ctypes.byref(p), ctypes.byref(t), kw.get("k", FAKE),
+                                                      kw.get("v", FAKE), count, None)
+    assert call(t, count=97) == CAPACITY
+    assert call(t, count=0) == INVALID
+    assert call(t, count=-3) == INVALID
+    assert call(t, k=0) == INVALID
+    assert call(t, v=FAKE + 8) == INVALID
+    assert call(_tree(length=4000, k_node=0)) == INVALID
+    assert lib.recsa_append(ctypes.byref(_p(top_k=-1)), ctypes.byref(t), FAKE, FAKE, 1, None) == INVALID
     assert t.length == 4000  # unchanged on failure
 
 
