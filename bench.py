@@ -485,6 +485,17 @@ def run_profile_case(args):
         R.check_device_errors(ws)
         print(json.dumps({"profile": "prefill", "length": w.length, "chunk": w.chunk,
                           "tiles": w.batch * w.kv_heads * w.chunk, "kernel_source_sha256": kernel_source_sha()}))
+    elif args.profile == "append":
+        w = dataclasses.replace(I.WORKLOADS["decode_1m"], batch=1, kv_heads=4, q_heads=16)
+        inp = I.decode_inputs(w, device="cuda", capacity=w.length + 64)
+        p = R.params(num_kv_heads=w.kv_heads, num_q_heads=w.q_heads, branching=w.branching, top_k=w.top_k)
+        tree, ws = make_tree(R, p, inp, w.length)
+        g = torch.Generator(device="cuda").manual_seed(7)
+        kn, vn = (torch.randn(1, 1, w.kv_heads, 128, generator=g, device="cuda").to(torch.bfloat16) for _ in range(2))
+        for _ in range(6):  # one token a step, the cache growing as in a decode loop
+            R.append(p, tree, kn, vn)
+        torch.cuda.synchronize()
+        print(json.dumps({"profile": "append", "length": tree.length, "kv_heads": w.kv_heads}))
     elif args.profile == "build":
         w = dataclasses.replace(I.WORKLOADS["build_decode_2m"], length=1 << 19)
         inp = I.decode_inputs(w, device="cuda")
@@ -589,7 +600,7 @@ def main():
     ap.add_argument("--headline-only", action="store_true", help="skip the prefill and build legs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--profile", choices=["decode", "prefill", "build"], help="run a small case of one kernel for ncu")
+    ap.add_argument("--profile", choices=["decode", "prefill", "build", "append"], help="run a small case of one kernel for ncu")
     args = ap.parse_args()
     if args.profile:
         run_profile_case(args)
