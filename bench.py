@@ -198,8 +198,13 @@ def decode_entries(R, p, tree, ws, q):
     return int(ent.sum().item())
 
 
-def leg_decode_1m(R, timer, args, dist_on, hbm_peak, peaks_src):
+def leg_decode_1m(R, timer, args, dist_on, hbm_peak, peaks_src, heads=None):
+    """The headline decode.  heads = (h0, h1): this rank's block of KV heads of every
+    sequence (sharding by KV head); None: the whole batch (a replica)."""
     w = I.WORKLOADS["decode_1m"]
+    if heads is not None:
+        g = w.q_heads // w.kv_heads
+        w = dataclasses.replace(w, kv_heads=heads[1] - heads[0], q_heads=g * (heads[1] - heads[0]))
     inp = I.decode_inputs(w, device="cuda")
     p = R.params(num_kv_heads=w.kv_heads, num_q_heads=w.q_heads, branching=w.branching, top_k=w.top_k)
     tree, ws = make_tree(R, p, inp, w.length)
@@ -526,7 +531,11 @@ def run_gpu(args):
     timer = Timer(dist_on)
     visible = os.environ.get("CUDA_VISIBLE_DEVICES")
     clocks = ClockSampler(visible.split(",")[local].strip() if visible else local)
-    dec, w = leg_decode_1m(R, timer, args, dist_on, hbm_peak, peaks_src)
+    heads = None
+    if args.shard == "heads":
+        from hierarchical_sparse_attention_build_b200.sharding import kv_head_range
+        heads = kv_head_range(I.WORKLOADS["decode_1m"].kv_heads, rank, world)
+    dec, w = leg_decode_1m(R, timer, args, dist_on, hbm_peak, peaks_src, heads)
     extra = {}
     if not args.headline_only:
         extra["prefill"] = leg_prefill(R, timer, args, dist_on, hbm_peak, "prefill_524k", 524288)
@@ -549,7 +558,12 @@ def run_gpu(args):
         return
     B = w.batch
     n = world
-    value = n * dec["queries"] * args.steps / dec["total_s"]  # total_s is already the max over ranks
+    # total_s is already the max over ranks; replicas each decode their own batch, KV-head
+    # shards together decode one batch
+    shards = heads is not None
+    job_queries = dec["queries"] if shards else n * dec["queries"]
+    value = job_queries * args.steps / dec["total_s"]
+    w_all = I.WORKLOADS["decode_1m"]
     mean_s = dec["mean_s"]
     achieved = dec["bytes_per_launch"] / mean_s / 1e9
     traffic = recorded_traffic("decode_1m_attend_traffic")
@@ -562,21 +576,23 @@ def run_gpu(args):
         "warmup": args.warmup,
         "ms_per_step": mean_s * 1e3,
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if shards else "weak",
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": f"decode_1m: B={B}, L={w.length}, Hq={w.q_heads}, Hkv={w.kv_heads}, d=128, "
+        "config": {"workload": f"decode_1m: B={B}, L={w.length}, Hq={w_all.q_heads}, Hkv={w_all.kv_heads}, d=128, "
                                f"b={w.branching}, k={w.top_k}, Q=1 query per sequence, needles=64 (bf16 K/V, "
                                "fp32 accumulation, bf16 output)",
-                   "global_batch": B * n, "seq_len": w.length, "parallelism": f"replicas x{n} (no collective)",
+                   "global_batch": B if shards else B * n, "seq_len": w.length,
+                   "parallelism": (f"KV-head shards x{n}, {w.kv_heads} KV heads on rank 0 (no collective)" if shards
+                                   else f"replicas x{n} (no collective)"),
                    "l2": "flushed between timed steps (256 MiB write, untimed)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": traffic,
                      "kernel": "attend_lean_kernel<4,4,2> (recsa_decode, 4-CTA clusters)",
                      "algorithmic_bytes_per_launch": dec["bytes_per_launch"],
                      "peak_source": f"{peaks_src} hbm_gbs (MEASURED_PEAKS.json)"},
-        "e2e": {"value": n * dec["queries"] * args.steps / dec["e2e_total_s"], "unit": "queries/s",
+        "e2e": {"value": job_queries * args.steps / dec["e2e_total_s"], "unit": "queries/s",
                 "h2d_bytes_per_step": dec["h2d"], "d2h_bytes_per_step": dec["d2h"]},
         "gpu_launches": args.steps,
         "clocks": clk,
@@ -600,6 +616,9 @@ def main():
     ap.add_argument("--headline-only", action="store_true", help="skip the prefill and build legs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--shard", default="sequences", choices=["sequences", "heads"],
+                    help="with N GPUs: N replicas of the batch (sequences, weak scaling) or the batch's "
+                         "KV heads split over the N GPUs (heads, strong scaling)")
     ap.add_argument("--profile", choices=["decode", "prefill", "build", "append"], help="run a small case of one kernel for ncu")
     args = ap.parse_args()
     if args.profile:
