@@ -62,6 +62,7 @@ class Tree(ctypes.Structure):
         ("k_node", ctypes.c_void_p),
         ("v_node", ctypes.c_void_p),
         ("pooler", ctypes.c_void_p),
+        ("seq_len", ctypes.c_void_p),
     ]
 
 
@@ -153,7 +154,10 @@ class RecsaTree:
     """A layer's token caches plus its node arena (torch tensors) and the C struct over them."""
 
     def __init__(self, p: Params, k_tok: torch.Tensor, v_tok: torch.Tensor, pooler: torch.Tensor, length: int,
-                 k_node: torch.Tensor | None = None, v_node: torch.Tensor | None = None):
+                 k_node: torch.Tensor | None = None, v_node: torch.Tensor | None = None,
+                 seq_len: torch.Tensor | None = None):
+        """seq_len: optional int64 [batch] device tensor of per-sequence lengths (length is then
+        the longest); the library advances it on the device when it appends."""
         assert k_tok.dtype == torch.bfloat16 and v_tok.dtype == torch.bfloat16 and pooler.dtype == torch.float32
         assert k_tok.is_contiguous() and v_tok.is_contiguous() and pooler.is_contiguous()
         batch, hkv, capacity, d = k_tok.shape
@@ -165,8 +169,11 @@ class RecsaTree:
             v_node = torch.empty_like(k_node)
         self.k_tok, self.v_tok, self.k_node, self.v_node, self.pooler = k_tok, v_tok, k_node, v_node, pooler
         self.node_rows = rows
+        if seq_len is not None:
+            assert seq_len.dtype == torch.int64 and seq_len.is_contiguous() and seq_len.numel() == batch
+        self.seq_len = seq_len
         self.c = Tree(batch, 0, capacity, length, k_tok.data_ptr(), v_tok.data_ptr(), k_node.data_ptr(),
-                      v_node.data_ptr(), pooler.data_ptr())
+                      v_node.data_ptr(), pooler.data_ptr(), seq_len.data_ptr() if seq_len is not None else None)
 
     @property
     def length(self) -> int:

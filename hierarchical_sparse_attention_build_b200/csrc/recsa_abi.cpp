@@ -140,6 +140,8 @@ recsa_status check_tree(const recsa_params *p, const recsa_tree *t, TreeGeom *g)
     if (!ptrs[i]) return fail(RECSA_ERR_INVALID_ARGUMENT, "tree->%s is NULL", names[i]);
     if (!aligned16(ptrs[i])) return fail(RECSA_ERR_INVALID_ARGUMENT, "tree->%s is not 16-byte aligned", names[i]);
   }
+  if (t->seq_len && reinterpret_cast<uintptr_t>(t->seq_len) % 8 != 0)
+    return fail(RECSA_ERR_INVALID_ARGUMENT, "tree->seq_len is not 8-byte aligned");
   return RECSA_OK;
 }
 
@@ -175,11 +177,12 @@ recsa_status build_range(const TreeGeom &g, const recsa_tree &t, int64_t length,
   return RECSA_OK;
 }
 
-// Appends `chunk` tokens at L and rebuilds every node whose span meets them.  When the chunk
-// is short and each level has at most kPathNodes such nodes per (sequence, head) (a decode
-// step's token, a short prefill chunk), one launch appends and walks the ancestor path, a
-// warp per (sequence, head); otherwise the tokens are copied and each level is rebuilt by
-// its own launch, wide over the level's nodes.
+// Appends `chunk` tokens at L (at each sequence's own length when the tree has per-sequence
+// lengths) and rebuilds every node whose span meets them.  When the chunk is short and each
+// level has at most kPathNodes such nodes per (sequence, head) (a decode step's token, a
+// short prefill chunk), or when the sequences have their own lengths, one launch appends
+// and walks the ancestor path, a CTA per (sequence, head); otherwise the tokens are copied
+// and each level is rebuilt by its own launch, wide over the level's nodes.
 constexpr int64_t kPathNodes = 4;
 constexpr int kPathTokens = 64;
 recsa_status extend_tree(const TreeGeom &g, const recsa_tree &t, const void *k_new, const void *v_new, int64_t L,
@@ -187,15 +190,11 @@ recsa_status extend_tree(const TreeGeom &g, const recsa_tree &t, const void *k_n
   const int64_t L2 = L + chunk;
   const int T_new = levels_for(L2, g.b);
   const int T_old = levels_for(L, g.b);
-  int64_t j0[kMaxLevels + 1] = {0}, j1[kMaxLevels + 1] = {0};
   int64_t most = 0;
-  for (int l = 1; l <= T_new; ++l) {
-    j0[l] = l <= T_old ? L / g.span[l] : 0;
-    j1[l] = ceil_div(L2, g.span[l]);
-    most = std::max(most, j1[l] - j0[l]);
-  }
-  if (chunk <= kPathTokens && most <= kPathNodes) {
-    const int rc = launch_extend(g, t, k_new, v_new, L, chunk, T_new, j0, j1, stream);
+  for (int l = 1; l <= T_new; ++l)
+    most = std::max(most, ceil_div(L2, g.span[l]) - (l <= T_old ? L / g.span[l] : 0));
+  if (t.seq_len || (chunk <= kPathTokens && most <= kPathNodes)) {
+    const int rc = launch_extend(g, t, k_new, v_new, L, chunk, T_new, stream);
     return rc != 0 ? cuda_fail(rc, "append and path update") : RECSA_OK;
   }
   const int rc = launch_append(g, t, k_new, v_new, L, chunk, stream);
@@ -380,6 +379,10 @@ RECSA_API recsa_status recsa_append(const recsa_params *params, recsa_tree *tree
                 (long long)tree->capacity);
   s = extend_tree(g, *tree, k_new, v_new, L, count, stream);
   if (s != RECSA_OK) return s;
+  if (tree->seq_len) {
+    const int rc = launch_advance_lengths(tree->seq_len, tree->batch, count, stream);
+    if (rc != 0) return cuda_fail(rc, "advance of the sequence lengths");
+  }
   tree->length = L + count;
   return RECSA_OK;
 }
@@ -432,8 +435,12 @@ RECSA_API recsa_status recsa_prefill_chunk(const recsa_params *params, recsa_tre
   l.cluster_size = debug ? debug->cluster_size : 0;
   l.kernel = debug ? debug->kernel : 0;
   l.debug = debug;
-  const int rc = launch_attend(l, stream);
+  int rc = launch_attend(l, stream);
   if (rc != 0) return cuda_fail(rc, "prefill attend");
+  if (tree->seq_len) {
+    rc = launch_advance_lengths(tree->seq_len, tree->batch, chunk, stream);
+    if (rc != 0) return cuda_fail(rc, "advance of the sequence lengths");
+  }
   tree->length = L2;
   return RECSA_OK;
 }

@@ -61,8 +61,9 @@ struct AttendArgs {
   WsHeader *hdr;
   int32_t *sel_idx;
   int32_t *entries;
+  const int64_t *seq_len;  // per-sequence lengths (NULL: every sequence has `length`)
   int64_t cap;
-  int64_t length;  // decode: L; prefill: L before the chunk
+  int64_t length;  // decode: L; prefill: L before the chunk (the longest, with seq_len)
   int64_t row_off[kMaxLevels + 1];
   int64_t slots[kMaxLevels + 1];
   int32_t span[kMaxLevels + 1];   // b^l, saturated above any capacity
@@ -115,7 +116,9 @@ __device__ __forceinline__ TileInfo tile_info(const AttendArgs &a, const Geo &ge
   const int sg = tile / a.nq;
   t.g = sg % a.hkv;
   t.s = sg / a.hkv;
-  t.p = (int)(a.causal ? a.length + t.qi : a.length);
+  // a sequence's own length, held to [0, length] (the workspace check flags an entry outside)
+  const int64_t len = a.seq_len ? min(max(a.seq_len[t.s], (int64_t)0), a.length) : a.length;
+  t.p = (int)(a.causal ? len + t.qi : len);
   t.bh = (int64_t)t.s * a.hkv + t.g;
   // levels above the tokens: ceil(p / b^T) <= b  <=>  p <= b^(T+1), so T = #{l >= 1 : b^l < p}
   int T = 0;
@@ -124,12 +127,17 @@ __device__ __forceinline__ TileInfo tile_info(const AttendArgs &a, const Geo &ge
   return t;
 }
 
+// Nodes of a level whose nodes span `span` tokens, over `p` tokens: ceil(p / span).
+__device__ __forceinline__ int nodes_at(int p, int span) {
+  return (int)(((uint32_t)p + (uint32_t)span - 1u) / (uint32_t)span);  // p < 2^31, span <= 2^30 + 1
+}
+
 // Candidate count of the top level; *forced_pos = position of the forced partial node or -1.
 __device__ __forceinline__ int top_candidates(const AttendArgs &a, const Geo &geo, const TileInfo &t,
                                               int *forced_pos) {
   *forced_pos = -1;
   if (t.T == 0) return t.p;
-  if (!a.causal) return geo.nlen[t.T];
+  if (!a.causal) return a.seq_len ? nodes_at(t.p, geo.span[t.T]) : geo.nlen[t.T];
   const int full = t.p / geo.span[t.T];
   if (t.p - full * geo.span[t.T]) {
     *forced_pos = full;
@@ -164,7 +172,10 @@ __device__ __forceinline__ int child_count(const AttendArgs &a, const Geo &geo, 
                                            bool *last_forced) {
   const int node = (int)(v & kNodeMask);
   *last_forced = false;
-  if (!a.causal) return max(0, min(a.b, geo.nlen[lvl - 1] - node * a.b));
+  if (!a.causal) {
+    const int nlen = a.seq_len ? nodes_at(p, geo.span[lvl - 1]) : geo.nlen[lvl - 1];
+    return max(0, min(a.b, nlen - node * a.b));
+  }
   if (!(v & kForced)) return a.b;
   const int sb = geo.span[lvl - 1];
   const int first = node * a.b;  // children starting before p are visible
@@ -1795,6 +1806,13 @@ __global__ void __launch_bounds__(kWarpKernelMaxWarps * 32, (G <= 4 ? 2 : 1)) at
 
 // ================================================================== launch
 
+// Flags per-sequence lengths outside [0, length] in the workspace error word (the attend
+// kernels clamp them into that range).
+__global__ void check_lengths_kernel(const int64_t *seq_len, int batch, int64_t length, WsHeader *hdr) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < batch && (seq_len[i] < 0 || seq_len[i] > length)) atomicOr(&hdr->err, kErrIndex);
+}
+
 int sm_count_cached() {
   int dev = 0, n = 148;
   cudaGetDevice(&dev);
@@ -1918,6 +1936,13 @@ int launch_g(const AttendArgs &a, int kernel, int CS, cudaStream_t stream) {
 }  // namespace
 
 int launch_attend(const AttendLaunch &l, void *stream) {
+  if (l.tree.seq_len) {
+    const int threads = 128;
+    check_lengths_kernel<<<(l.geom.batch + threads - 1) / threads, threads, 0, (cudaStream_t)stream>>>(
+        l.tree.seq_len, l.geom.batch, l.length, reinterpret_cast<WsHeader *>(l.ws));
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return (int)e;
+  }
   AttendArgs a = {};
   a.k_tok = reinterpret_cast<const uint16_t *>(l.tree.k_tok);
   a.v_tok = reinterpret_cast<const uint16_t *>(l.tree.v_tok);
@@ -1932,6 +1957,7 @@ int launch_attend(const AttendLaunch &l, void *stream) {
   a.entries = l.debug ? l.debug->entries : nullptr;
   a.cap = l.geom.capacity;
   a.length = l.length;
+  a.seq_len = l.tree.seq_len;
   for (int i = 0; i <= kMaxLevels; ++i) {
     a.row_off[i] = l.geom.row_off[i];
     a.slots[i] = l.geom.slots[i];

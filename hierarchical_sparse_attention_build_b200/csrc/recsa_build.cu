@@ -42,6 +42,9 @@ struct BuildArgs {
   int64_t j0, nj;         // nodes [j0, j0 + nj) of level l, for every (sequence, head)
   int32_t b;
   int32_t bh;             // batch * Hkv
+  int32_t hkv;
+  int64_t span;           // tokens under a level l node (b^l)
+  const int64_t *seq_len; // per-sequence lengths (NULL: every sequence has `length`)
   const float *pooler;    // [128][128] row-major W
 };
 
@@ -186,19 +189,29 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_level_kernel(const Bui
   const int64_t total = (int64_t)a.bh * a.nj;
   for (int64_t base = (int64_t)blockIdx.x * kNodesPerBlock; base < total;
        base += (int64_t)gridDim.x * kNodesPerBlock) {
+    bool live[NPW];
     for (int t = 0; t < NPW; ++t) {
       const int nl = warp * NPW + t;
       const int64_t id = base + nl;
       float ks[4] = {0.f, 0.f, 0.f, 0.f}, vs[4] = {0.f, 0.f, 0.f, 0.f};
-      if (id < total) {
+      live[t] = id < total;
+      if (live[t]) {
         const int64_t bhi = id / a.nj;
         const int64_t j = a.j0 + id % a.nj;
-        const int64_t c0 = j * a.b;
-        const int64_t c1 = min(c0 + (int64_t)a.b, a.n_prev);
-        const uint16_t *kb = a.src_k + (a.src_row_off + bhi * a.src_slots) * kD + lane * 4;
-        const uint16_t *vb = a.src_v + (a.src_row_off + bhi * a.src_slots) * kD + lane * 4;
-        node_means<true>(kb, vb, c0, c1, a.n_prev, a.length, a.span_prev, ks, vs);
-        store_row4(a.dst_v + (a.dst_row_off + bhi * a.dst_slots + j) * kD + lane * 4, vs);
+        int64_t length = a.length, n_prev = a.n_prev;
+        if (a.seq_len) {  // this sequence's own length: its level has ceil(len / b^l) nodes
+          length = min(max(a.seq_len[bhi / a.hkv], (int64_t)0), a.length);
+          n_prev = (length + a.span_prev - 1) / a.span_prev;
+          live[t] = j < (length + a.span - 1) / a.span;
+        }
+        if (live[t]) {
+          const int64_t c0 = j * a.b;
+          const int64_t c1 = min(c0 + (int64_t)a.b, n_prev);
+          const uint16_t *kb = a.src_k + (a.src_row_off + bhi * a.src_slots) * kD + lane * 4;
+          const uint16_t *vb = a.src_v + (a.src_row_off + bhi * a.src_slots) * kD + lane * 4;
+          node_means<true>(kb, vb, c0, c1, n_prev, length, a.span_prev, ks, vs);
+          store_row4(a.dst_v + (a.dst_row_off + bhi * a.dst_slots + j) * kD + lane * 4, vs);
+        }
       }
       *reinterpret_cast<float4 *>(Mean + nl * kD + lane * 4) = make_float4(ks[0], ks[1], ks[2], ks[3]);
     }
@@ -209,7 +222,7 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_level_kernel(const Bui
 #pragma unroll
     for (int n = 0; n < NPW; ++n) {
       const int64_t id = base + warp * NPW + n;
-      if (id < total) {
+      if (live[n]) {
         const int64_t bhi = id / a.nj;
         const int64_t j = a.j0 + id % a.nj;
         store_row4(a.dst_k + (a.dst_row_off + bhi * a.dst_slots + j) * kD + lane * 4, acc[n]);
@@ -235,14 +248,13 @@ struct ExtendArgs {
   uint16_t *k_tok, *v_tok;      // [B][Hkv][capacity][128]
   uint16_t *k_node, *v_node;    // node arena
   const float *pooler;
+  const int64_t *seq_len;       // per-sequence lengths before the append (NULL: all `at`)
   int64_t capacity;
-  int64_t at;                   // first new slot (the length before the append)
-  int64_t length;               // length after it
-  int32_t chunk, hkv, b, levels;  // levels = T(length)
+  int64_t at;                   // first new slot (the length before the append; the longest one)
+  int32_t chunk, hkv, b, levels;  // levels = T(at + chunk)
   int64_t row_off[kMaxLevels + 1];
   int64_t slots[kMaxLevels + 1];
   int64_t span[kMaxLevels + 1];
-  int64_t j0[kMaxLevels + 1], j1[kMaxLevels + 1];  // nodes rebuilt at level l
 };
 constexpr int kExtendThreads = 2 * kD;  // one thread per key dimension and per value dimension
 constexpr int kHalfK = kD / 2;          // W columns held by each thread of a dimension
@@ -263,6 +275,18 @@ __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendA
   const int64_t bhi = blockIdx.x;   // (sequence, head)
   const int d = tid & (kD - 1);
   const bool is_v = tid >= kD;
+  // this sequence's length before (at) and after (length) the append, and its levels
+  const int64_t at = a.seq_len ? min(max(a.seq_len[bhi / a.hkv], (int64_t)0), a.at) : a.at;
+  const int64_t length = at + a.chunk;
+  int t_old = 0, t_new = 0;  // T(n) = #{l >= 1 : b^l < n}
+  while (t_new < a.levels && a.span[t_new + 1] < length) ++t_new;
+  while (t_old < t_new && a.span[t_old + 1] < at) ++t_old;
+  // level l rebuilds nodes [j0, j1): those whose spans meet the new tokens (a level that
+  // becomes new is built whole)
+  auto node_range = [&](int l, int64_t *j0, int64_t *j1) {
+    *j0 = l <= t_old ? at / a.span[l] : 0;
+    *j1 = (length + a.span[l] - 1) / a.span[l];
+  };
 
   // W in flight (a warp reads one 512-byte row) while the tokens are appended and the first
   // children load
@@ -272,8 +296,8 @@ __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendA
   for (int i = 0; i < kPieces; ++i) w[i] = __ldg(reinterpret_cast<const float4 *>(a.pooler) + tid + i * kExtendThreads);
   {
     const int64_t s = bhi / a.hkv, h = bhi % a.hkv;
-    uint4 *kt = reinterpret_cast<uint4 *>(a.k_tok + (bhi * a.capacity + a.at) * kD);
-    uint4 *vt = reinterpret_cast<uint4 *>(a.v_tok + (bhi * a.capacity + a.at) * kD);
+    uint4 *kt = reinterpret_cast<uint4 *>(a.k_tok + (bhi * a.capacity + at) * kD);
+    uint4 *vt = reinterpret_cast<uint4 *>(a.v_tok + (bhi * a.capacity + at) * kD);
     for (int e = tid; e < a.chunk * 16; e += kExtendThreads) {  // 16 pieces a row
       const int64_t src = ((s * a.chunk + (e >> 4)) * a.hkv + h) * 16 + (e & 15);
       kt[e] = __ldg(a.k_new + src);
@@ -282,9 +306,11 @@ __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendA
   }
   // every child row the walk reads above level 1, into L2 ahead of the dependent levels
   // (K and V, two 128-byte lines each)
-  for (int l = 2; l <= a.levels; ++l) {
-    const int64_t n_prev = (a.length + a.span[l - 1] - 1) / a.span[l - 1];
-    const int64_t c0 = a.j0[l] * a.b, c1 = min(a.j1[l] * a.b, n_prev);
+  for (int l = 2; l <= t_new; ++l) {
+    const int64_t n_prev = (length + a.span[l - 1] - 1) / a.span[l - 1];
+    int64_t j0, j1;
+    node_range(l, &j0, &j1);
+    const int64_t c0 = j0 * a.b, c1 = min(j1 * a.b, n_prev);
     const int64_t base = (a.row_off[l - 1] + bhi * a.slots[l - 1]) * kD;
     for (int64_t e = tid; e < (c1 - c0) * 4; e += kExtendThreads)
       prefetch_l2(((e & 2) ? a.v_node : a.k_node) + base + (c0 + (e >> 2)) * kD + (e & 1) * (kD / 2));
@@ -294,14 +320,16 @@ __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendA
   float wr[kHalfK];  // W[d][64 * is_v + i]
   bool w_ready = false;
   const int kbase = is_v ? kHalfK : 0;
-  for (int l = 1; l <= a.levels; ++l) {
+  for (int l = 1; l <= t_new; ++l) {
     const int64_t span_prev = a.span[l - 1];
-    const int64_t n_prev = (a.length + span_prev - 1) / span_prev;
+    const int64_t n_prev = (length + span_prev - 1) / span_prev;
+    int64_t j0, j1;
+    node_range(l, &j0, &j1);
     const uint16_t *src = l == 1 ? (is_v ? a.v_tok : a.k_tok) + bhi * a.capacity * kD
                                  : (is_v ? a.v_node : a.k_node) + (a.row_off[l - 1] + bhi * a.slots[l - 1]) * kD;
     uint16_t *dk = a.k_node + (a.row_off[l] + bhi * a.slots[l]) * kD;
     uint16_t *dv = a.v_node + (a.row_off[l] + bhi * a.slots[l]) * kD;
-    for (int64_t j = a.j0[l]; j < a.j1[l]; ++j) {
+    for (int64_t j = j0; j < j1; ++j) {
       const int64_t c0 = j * a.b, c1 = min(c0 + (int64_t)a.b, n_prev);
       float sum = 0.f;
 #pragma unroll 16
@@ -310,7 +338,7 @@ __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendA
       if (is_v) {  // token-weighted: the level's last child gets its share tokens / span_prev
         float wsum = nch;
         if (c1 == n_prev && c1 > c0) {
-          const int64_t last_tokens = a.length - (c1 - 1) * span_prev;
+          const int64_t last_tokens = length - (c1 - 1) * span_prev;
           if (last_tokens < span_prev) {
             const float f1 = (float)last_tokens / (float)span_prev - 1.f;
             sum = __fmaf_rn(f1, bf16_lo(src[(c1 - 1) * kD + d]), sum);
@@ -470,6 +498,9 @@ int launch_build_level(const TreeGeom &g, const recsa_tree &t, int level, int64_
   a.nj = j1 - j0;
   a.b = g.b;
   a.bh = g.batch * g.hkv;
+  a.hkv = g.hkv;
+  a.span = g.span[level];
+  a.seq_len = t.seq_len;
   a.pooler = t.pooler;
   const int rc = configure_smem();
   if (rc != 0) return rc;
@@ -487,7 +518,7 @@ int launch_build_level(const TreeGeom &g, const recsa_tree &t, int level, int64_
 }
 
 int launch_extend(const TreeGeom &g, const recsa_tree &t, const void *k_new, const void *v_new, int64_t at,
-                  int chunk, int levels, const int64_t *j0, const int64_t *j1, void *stream) {
+                  int chunk, int levels, void *stream) {
   ExtendArgs a;
   a.k_new = reinterpret_cast<const uint4 *>(k_new);
   a.v_new = reinterpret_cast<const uint4 *>(v_new);
@@ -496,9 +527,9 @@ int launch_extend(const TreeGeom &g, const recsa_tree &t, const void *k_new, con
   a.k_node = reinterpret_cast<uint16_t *>(t.k_node);
   a.v_node = reinterpret_cast<uint16_t *>(t.v_node);
   a.pooler = t.pooler;
+  a.seq_len = t.seq_len;
   a.capacity = g.capacity;
   a.at = at;
-  a.length = at + chunk;
   a.chunk = chunk;
   a.hkv = g.hkv;
   a.b = g.b;
@@ -507,13 +538,22 @@ int launch_extend(const TreeGeom &g, const recsa_tree &t, const void *k_new, con
     a.row_off[l] = g.row_off[l];
     a.slots[l] = g.slots[l];
     a.span[l] = g.span[l];
-    a.j0[l] = l <= levels ? j0[l] : 0;
-    a.j1[l] = l <= levels ? j1[l] : 0;
   }
   const int rc = configure_smem();
   if (rc != 0) return rc;
   const int64_t grid = (int64_t)g.batch * g.hkv;
   extend_kernel<<<(unsigned)grid, kExtendThreads, kExtendSmem, (cudaStream_t)stream>>>(a);
+  return (int)cudaGetLastError();
+}
+
+__global__ void advance_lengths_kernel(int64_t *seq_len, int batch, int64_t count) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < batch) seq_len[i] += count;
+}
+
+int launch_advance_lengths(int64_t *seq_len, int batch, int64_t count, void *stream) {
+  const int threads = 128;
+  advance_lengths_kernel<<<(batch + threads - 1) / threads, threads, 0, (cudaStream_t)stream>>>(seq_len, batch, count);
   return (int)cudaGetLastError();
 }
 

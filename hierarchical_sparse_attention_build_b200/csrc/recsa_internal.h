@@ -55,10 +55,13 @@ int launch_build_level(const TreeGeom &g, const recsa_tree &t, int level, int64_
                        void *stream);
 int launch_append(const TreeGeom &g, const recsa_tree &t, const void *k_new, const void *v_new, int64_t at,
                   int chunk, void *stream);
-// Append `chunk` tokens at slot `at` and rebuild nodes [j0[l], j1[l]) of levels 1..levels in
-// one launch (one warp per (sequence, head) walks up the levels).
+// Append `chunk` tokens at slot `at` (at t.seq_len[s] when the tree has per-sequence lengths)
+// and rebuild the nodes over them, all levels in one launch (a CTA per (sequence, head)
+// walks up the levels).  levels = T of the longest new length.
 int launch_extend(const TreeGeom &g, const recsa_tree &t, const void *k_new, const void *v_new, int64_t at,
-                  int chunk, int levels, const int64_t *j0, const int64_t *j1, void *stream);
+                  int chunk, int levels, void *stream);
+// seq_len[s] += count for every sequence (queued after the kernels that read the old lengths).
+int launch_advance_lengths(int64_t *seq_len, int batch, int64_t count, void *stream);
 
 struct AttendLaunch {
   TreeGeom geom;

@@ -97,7 +97,17 @@ typedef struct recsa_params {
  *                  sequence s, KV head h, node j sits at row
  *                  level_row_offsets[l] + (s*Hkv + h) * ceil(capacity / b^l) + j.
  *   pooler       : fp32 [128][128] row-major W (node key = W @ mean of child keys).
- * All sequences share `length`. */
+ *   seq_len      : NULL when every sequence holds `length` tokens.  Otherwise a device
+ *                  array int64 [batch], 8-byte aligned, owned by the caller: sequence s
+ *                  holds seq_len[s] tokens, 0 <= seq_len[s] <= length, and `length` is
+ *                  the longest (the host-side bound every size check uses).  Each
+ *                  sequence then has its own tree over its own tokens (levels, node
+ *                  counts, query positions).  recsa_append and recsa_prefill_chunk append
+ *                  at each sequence's own end and advance seq_len on the device (queued
+ *                  after their kernels) as they advance `length` on the host.  The
+ *                  kernels clamp an entry outside [0, length] into it; decode and prefill
+ *                  calls also flag one in the workspace error word
+ *                  (RECSA_ERR_DEVICE_CHECK from recsa_check_device_errors). */
 typedef struct recsa_tree {
   int32_t batch;
   int32_t reserved;
@@ -108,6 +118,7 @@ typedef struct recsa_tree {
   void *k_node;
   void *v_node;
   const float *pooler;
+  int64_t *seq_len;
 } recsa_tree;
 
 /* Optional diagnostics and launch-shape overrides of recsa_decode / recsa_prefill_chunk

@@ -5,7 +5,8 @@
 // accesses (with AddressSanitizer) and its results, without a GPU.
 //
 // usage: emu_lean <case dir>
-//   <dir>/params.txt  key value lines (scalars) and "row_off"/"slots" lines (kMaxLevels+1 ints)
+//   <dir>/params.txt  key value lines (scalars), "row_off"/"slots" lines (kMaxLevels+1 ints) and
+//                     an optional "seq_len" line (one length per sequence)
 //   <dir>/{k_tok,v_tok,k_node,v_node,q}.bin  bf16 arrays in the library's layouts
 //   writes <dir>/{out,sel,entries}.bin and <dir>/err.txt (the workspace error word)
 #include <fstream>
@@ -112,7 +113,7 @@ int main(int argc, char **argv) {
   }
   const std::string dir = argv[1];
   std::map<std::string, double> kv;
-  std::vector<int64_t> row_off, slots;
+  std::vector<int64_t> row_off, slots, seq_len;
   {
     std::ifstream f(dir + "/params.txt");
     std::string line;
@@ -120,9 +121,9 @@ int main(int argc, char **argv) {
       std::istringstream ss(line);
       std::string key;
       ss >> key;
-      if (key == "row_off" || key == "slots") {
+      if (key == "row_off" || key == "slots" || key == "seq_len") {
         int64_t x;
-        auto &dst = key == "row_off" ? row_off : slots;
+        auto &dst = key == "row_off" ? row_off : key == "slots" ? slots : seq_len;
         while (ss >> x) dst.push_back(x);
       } else {
         double x;
@@ -169,6 +170,7 @@ int main(int argc, char **argv) {
   a.sel_idx = (top_k >= 1 && top_k <= 64) ? sel.data() : nullptr;
   a.sel_levels = sel_levels;
   a.entries = ent.data();
+  a.seq_len = seq_len.empty() ? nullptr : seq_len.data();
   a.cap = (int64_t)kv["cap"];
   a.length = (int64_t)kv["length"];
   for (int i = 0; i <= kMaxLevels; ++i) {

@@ -175,6 +175,7 @@ def test_append_capacity_and_arguments_rejected():
     assert call(t, k=0) == INVALID
     assert call(t, v=FAKE + 8) == INVALID
     assert call(_tree(length=4000, k_node=0)) == INVALID
+    assert call(_tree(length=4000, seq_len=FAKE + 4)) == INVALID  # per-sequence lengths need 8-byte alignment
     assert lib.recsa_append(ctypes.byref(_p(top_k=-1)), ctypes.byref(t), FAKE, FAKE, 1, None) == INVALID
     assert t.length == 4000  # unchanged on failure
 

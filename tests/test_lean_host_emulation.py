@@ -58,8 +58,9 @@ def _rph(G, CS, max_cand):
     raise ValueError("no lean shape")
 
 
-def _run(emu_bin, tmp_path, B, hkv, G, L, b, k, Q, CS, causal=False, seed=1):
-    """Lay out the oracle's bf16 tree, run the kernel on host threads, check every tile."""
+def _run(emu_bin, tmp_path, B, hkv, G, L, b, k, Q, CS, causal=False, seed=1, lens=None):
+    """Lay out the oracle's bf16 tree, run the kernel on host threads, check every tile.
+    lens: per-sequence lengths (decode; L is then their maximum)."""
     C = Q if causal else 0
     cap = L + C
     inp = I.random_case(B, L, hkv, hkv * G, Q, seed=seed, capacity=cap, chunk=C)
@@ -71,7 +72,11 @@ def _run(emu_bin, tmp_path, B, hkv, G, L, b, k, Q, CS, causal=False, seed=1):
         kb, vb = kb[:, :, :cap], vb[:, :, :cap]
         length_tree = L
     pooler = inp["pooler"].double().numpy()
-    trees = O.build_all(kb, vb, pooler, b, length_tree)
+    if lens is None:
+        trees = O.build_all(kb, vb, pooler, b, length_tree)
+    else:
+        trees = [[O.build_tree(O.bf16_bits_to_f64(kb[s, h, :n]), O.bf16_bits_to_f64(vb[s, h, :n]), pooler, b)
+                  if n else None for h in range(hkv)] for s, n in enumerate(lens)]
 
     p = R.params(num_kv_heads=hkv, num_q_heads=hkv * G, branching=b, top_k=k)
     node_rows, levels, offs = R.tree_layout(p, B, cap)
@@ -81,7 +86,7 @@ def _run(emu_bin, tmp_path, B, hkv, G, L, b, k, Q, CS, causal=False, seed=1):
     for s in range(B):
         for h in range(hkv):
             t = trees[s][h]
-            for lv in range(1, t.top + 1):
+            for lv in range(1, t.top + 1 if t is not None else 1):
                 n = t.keys[lv].shape[0]
                 r0 = offs[lv] + (s * hkv + h) * slots[lv]
                 knode[r0:r0 + n] = O.f64_to_bf16_bits(t.keys[lv])
@@ -100,13 +105,15 @@ def _run(emu_bin, tmp_path, B, hkv, G, L, b, k, Q, CS, causal=False, seed=1):
                top_k=k, sel_levels=sel_levels, cap=cap, length=L if causal else length_tree, b=b, levels=levels,
                hkv=hkv, nq=Q, causal=int(causal), table_rows_needed=mc + 1, max_cand=max_cand,
                scale=1.0 / math.sqrt(128.0))
-    d = tmp_path / f"case_{B}_{hkv}_{G}_{L}_{b}_{k}_{Q}_{CS}_{int(causal)}"
+    d = tmp_path / f"case_{B}_{hkv}_{G}_{L}_{b}_{k}_{Q}_{CS}_{int(causal)}_{int(lens is not None)}"
     d.mkdir()
     with open(d / "params.txt", "w") as f:
         for key, val in prm.items():
             f.write(f"{key} {val!r}\n")
         f.write("row_off " + " ".join(str(offs[i] if i <= levels else 0) for i in range(R.MAX_LEVELS + 1)) + "\n")
         f.write("slots " + " ".join(str(slots[i] if i <= levels else 0) for i in range(R.MAX_LEVELS + 1)) + "\n")
+        if lens is not None:
+            f.write("seq_len " + " ".join(str(n) for n in lens) + "\n")
     for name, arr in (("k_tok", ktok), ("v_tok", vtok), ("k_node", knode), ("v_node", vnode), ("q", bits(inp["q"]))):
         np.ascontiguousarray(arr, dtype=np.uint16).tofile(d / f"{name}.bin")
     r = subprocess.run([emu_bin, str(d)], capture_output=True, text=True, timeout=600)
@@ -122,7 +129,10 @@ def _run(emu_bin, tmp_path, B, hkv, G, L, b, k, Q, CS, causal=False, seed=1):
         for h in range(hkv):
             for qi in range(Q):
                 tile = (s * hkv + h) * Q + qi
-                pos = L + qi if causal else L
+                pos = L + qi if causal else (L if lens is None else lens[s])
+                if pos == 0:  # nothing visible: zeros
+                    assert not out[s, qi, h * G:(h + 1) * G].any()
+                    continue
                 top = len(O.level_counts(pos, b)) - 1
                 gsel = gpu_selection(sel, tile, top) if 1 <= k <= 64 else None
                 check_tile(stats, O.bf16_bits_to_f64(qb[s, qi, h * G:(h + 1) * G]), trees[s][h], pos, k, causal,
@@ -158,3 +168,9 @@ def test_causal_levels_past_128_candidates(emu_bin, tmp_path):
     # b = 16, k = 8, causal: up to 144 candidates a level, 3 rows per half-warp, and the
     # ranking by the generic count
     _run(emu_bin, tmp_path, 1, 1, 4, 3000, 16, 8, 6, 4, causal=True, seed=5)
+
+
+@pytest.mark.parametrize("CS", [2, 4])
+def test_decode_with_per_sequence_lengths(emu_bin, tmp_path, CS):
+    # an empty sequence, a single token, a shallow tree and the deepest one in one launch
+    _run(emu_bin, tmp_path, 4, 1, 4, 1000, 4, 2, 1, CS, lens=[0, 1, 37, 1000], seed=6)
