@@ -343,6 +343,34 @@ def leg_decode_loop(R, timer, args, dist_on):
                                           "attend (the partial node on the query's path always expanded)"}}
 
 
+def leg_decode_varlen(R, timer, args, dist_on):
+    """Decode over a batch of unequal sequences: 8 sequences of 8/8, 7/8, ..., 1/8 of 1M tokens
+    (the decode_1m head shape, b = 16, k = 8, one query each) in one call with per-sequence
+    lengths, next to the same batch with every sequence at 1M."""
+    w = dataclasses.replace(I.WORKLOADS["decode_1m"], batch=8)
+    inp = I.decode_inputs(w, device="cuda")
+    p = R.params(num_kv_heads=w.kv_heads, num_q_heads=w.q_heads, branching=w.branching, top_k=w.top_k)
+    lens = [w.length * (w.batch - i) // w.batch for i in range(w.batch)]
+    seq_len = torch.tensor(lens, dtype=torch.int64, device="cuda")
+    q = inp["q"]
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
+    steps = max(20, args.steps // 10) if not args.quick else 20
+    res = {"workload": f"decode_varlen: B={w.batch}, lengths {lens[-1]}..{lens[0]} (step {lens[0] - lens[1]}), "
+                       f"Hq={w.q_heads}, Hkv={w.kv_heads}, b={w.branching}, k={w.top_k}, 1 query per sequence"}
+    for name, sl in (("per_sequence_lengths", seq_len), ("all_at_1m", None)):
+        tree = R.RecsaTree(p, inp["k_tok"], inp["v_tok"], inp["pooler"], w.length, seq_len=sl)
+        ws = R.Workspace(p, tree.capacity, "cuda")
+        R.build_tree(p, tree)
+        per, _ = timer.run(lambda: R.decode(p, tree, q, out, ws), steps, 3)
+        t = max_over_ranks(sum(per), dist_on) / steps
+        R.check_device_errors(ws)
+        res[name] = {"queries_per_s": w.batch / t, "us_per_call": t * 1e6}
+        del tree, ws
+    del inp
+    torch.cuda.empty_cache()
+    return res
+
+
 def leg_build_2m(R, timer, args, dist_on, hbm_peak):
     w = I.WORKLOADS["build_decode_2m"]
     inp = I.decode_inputs(w, device="cuda")
@@ -542,6 +570,7 @@ def run_gpu(args):
         extra["prefill_1m"] = leg_prefill(R, timer, args, dist_on, hbm_peak, "prefill_1m", 1 << 20)
         extra["build_2m"] = leg_build_2m(R, timer, args, dist_on, hbm_peak)
         extra["decode_loop_1m"] = leg_decode_loop(R, timer, args, dist_on)
+        extra["decode_varlen"] = leg_decode_varlen(R, timer, args, dist_on)
     clk = clocks.stop()
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -63,6 +63,9 @@ class Tree(ctypes.Structure):
         ("v_node", ctypes.c_void_p),
         ("pooler", ctypes.c_void_p),
         ("seq_len", ctypes.c_void_p),
+        ("page_table", ctypes.c_void_p),
+        ("page_size", ctypes.c_int32),
+        ("num_pages", ctypes.c_int32),
     ]
 
 
@@ -155,13 +158,22 @@ class RecsaTree:
 
     def __init__(self, p: Params, k_tok: torch.Tensor, v_tok: torch.Tensor, pooler: torch.Tensor, length: int,
                  k_node: torch.Tensor | None = None, v_node: torch.Tensor | None = None,
-                 seq_len: torch.Tensor | None = None):
-        """seq_len: optional int64 [batch] device tensor of per-sequence lengths (length is then
+                 seq_len: torch.Tensor | None = None, page_table: torch.Tensor | None = None):
+        """k_tok, v_tok: contiguous caches [batch][Hkv][capacity][128], or with page_table (int32
+        [batch][pages per sequence] device tensor) a page pool [num_pages][Hkv][page_size][128].
+        seq_len: optional int64 [batch] device tensor of per-sequence lengths (length is then
         the longest); the library advances it on the device when it appends."""
         assert k_tok.dtype == torch.bfloat16 and v_tok.dtype == torch.bfloat16 and pooler.dtype == torch.float32
         assert k_tok.is_contiguous() and v_tok.is_contiguous() and pooler.is_contiguous()
-        batch, hkv, capacity, d = k_tok.shape
-        assert hkv == p.num_kv_heads and d == HEAD_DIM and v_tok.shape == k_tok.shape
+        assert v_tok.shape == k_tok.shape and k_tok.shape[3] == HEAD_DIM and k_tok.shape[1] == p.num_kv_heads
+        if page_table is None:
+            batch, _, capacity, _ = k_tok.shape
+            num_pages = page_size = 0
+        else:
+            assert page_table.dtype == torch.int32 and page_table.is_contiguous() and page_table.dim() == 2
+            num_pages, _, page_size, _ = k_tok.shape
+            batch = page_table.shape[0]
+            capacity = page_table.shape[1] * page_size
         self.p = p
         rows, self.levels, self.level_offsets = tree_layout(p, batch, capacity)
         if k_node is None:
@@ -172,8 +184,10 @@ class RecsaTree:
         if seq_len is not None:
             assert seq_len.dtype == torch.int64 and seq_len.is_contiguous() and seq_len.numel() == batch
         self.seq_len = seq_len
+        self.page_table = page_table
         self.c = Tree(batch, 0, capacity, length, k_tok.data_ptr(), v_tok.data_ptr(), k_node.data_ptr(),
-                      v_node.data_ptr(), pooler.data_ptr(), seq_len.data_ptr() if seq_len is not None else None)
+                      v_node.data_ptr(), pooler.data_ptr(), seq_len.data_ptr() if seq_len is not None else None,
+                      page_table.data_ptr() if page_table is not None else None, page_size, num_pages)
 
     @property
     def length(self) -> int:

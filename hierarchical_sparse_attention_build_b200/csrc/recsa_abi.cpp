@@ -142,6 +142,19 @@ recsa_status check_tree(const recsa_params *p, const recsa_tree *t, TreeGeom *g)
   }
   if (t->seq_len && reinterpret_cast<uintptr_t>(t->seq_len) % 8 != 0)
     return fail(RECSA_ERR_INVALID_ARGUMENT, "tree->seq_len is not 8-byte aligned");
+  if (t->page_table) {
+    const int32_t P = t->page_size;
+    if (P < 1 || P > 65536 || (P & (P - 1)) != 0)
+      return fail(RECSA_ERR_INVALID_ARGUMENT, "page_size %d is not a power of two in 1 .. 65536", P);
+    if (t->capacity % P != 0)
+      return fail(RECSA_ERR_INVALID_ARGUMENT, "capacity %lld is not a multiple of page_size %d",
+                  (long long)t->capacity, P);
+    if (t->num_pages < 1) return fail(RECSA_ERR_INVALID_ARGUMENT, "num_pages %d < 1", t->num_pages);
+    if (reinterpret_cast<uintptr_t>(t->page_table) % 4 != 0)
+      return fail(RECSA_ERR_INVALID_ARGUMENT, "tree->page_table is not 4-byte aligned");
+    if ((int64_t)t->num_pages * g->hkv * P > ((int64_t)1 << 40))
+      return fail(RECSA_ERR_UNSUPPORTED, "a page pool of %d pages", t->num_pages);
+  }
   return RECSA_OK;
 }
 

@@ -62,6 +62,8 @@ struct AttendArgs {
   int32_t *sel_idx;
   int32_t *entries;
   const int64_t *seq_len;  // per-sequence lengths (NULL: every sequence has `length`)
+  const int32_t *page_table;  // paged token caches: [B][cap >> page_shift] (NULL: contiguous)
+  int32_t page_shift, num_pages;
   int64_t cap;
   int64_t length;  // decode: L; prefill: L before the chunk (the longest, with seq_len)
   int64_t row_off[kMaxLevels + 1];
@@ -149,11 +151,31 @@ __device__ __forceinline__ int top_candidates(const AttendArgs &a, const Geo &ge
 struct LevelRows {
   const uint16_t *k, *v;
   int64_t nrows;
+  const int32_t *pages;  // level 0 of a paged cache: the sequence's page table (else NULL)
 };
 
+// Row of candidate `node` (node < nrows) relative to k / v: the node itself, or through the
+// page table at level 0 of a paged cache (pages are Hkv * page_size rows apart); -1 for a
+// page outside the pool.
+template <bool kPaged>
+__device__ __forceinline__ int64_t row_at(const AttendArgs &a, const LevelRows &lr, int64_t node) {
+  if (!kPaged || !lr.pages) return node;
+  const int pg = __ldg(lr.pages + (node >> a.page_shift));
+  if ((unsigned)pg >= (unsigned)a.num_pages) return -1;
+  return ((int64_t)pg * a.hkv << a.page_shift) + (node & ((int64_t(1) << a.page_shift) - 1));
+}
+
+template <bool kPaged>
 __device__ __forceinline__ LevelRows level_rows(const AttendArgs &a, const Geo &geo, int lvl, int64_t bh) {
   LevelRows r;
-  if (lvl == 0) {
+  r.pages = nullptr;
+  if (kPaged && lvl == 0) {  // head h's rows of page 0; pages are Hkv * page_size rows apart
+    const int64_t h = bh % a.hkv;
+    r.k = a.k_tok + (h << a.page_shift) * kD;
+    r.v = a.v_tok + (h << a.page_shift) * kD;
+    r.nrows = a.cap;
+    r.pages = a.page_table + (bh / a.hkv) * (a.cap >> a.page_shift);
+  } else if (lvl == 0) {
     r.k = a.k_tok + bh * a.cap * kD;
     r.v = a.v_tok + bh * a.cap * kD;
     r.nrows = a.cap;
@@ -543,7 +565,7 @@ __device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
-template <int G, int CS>
+template <int G, int CS, bool kPaged = false>
 __global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const AttendArgs a) {
   constexpr int RPH = (CS == 4 || G == 8) ? 2 : 4;  // rows per half-warp per pass (register budget)
   constexpr int PASS = kHalfWarps * RPH;              // rows per CTA per pass
@@ -597,19 +619,21 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const Attend
   // Gather rows [pass0, pass0 + PASS) of this CTA's slice [.., hi_r) of level lvl.  cl == nullptr
   // means the top level, whose position i is node i.
   auto gather = [&](RowSet<RPH> &rs, int lvl, const uint32_t *cl, int pass0, int hi_r, bool values) {
-    const LevelRows lr = level_rows(a, geo, lvl, t.bh);
+    const LevelRows lr = level_rows<kPaged>(a, geo, lvl, t.bh);
 #pragma unroll
     for (int r = 0; r < RPH; ++r) {
       const int i = pass0 + hw + kHalfWarps * r;
       rs.pos[r] = i;
       const uint32_t c = i < hi_r ? (cl ? cl[i] : ((uint32_t)i | (i == fpos ? kForced : 0u))) : kForced;
       const int64_t node = c & kNodeMask;
-      rs.ok[r] = i < hi_r && !(c & kForced) && node < lr.nrows;
-      if (i < hi_r && !(c & kForced) && node >= lr.nrows && j16 == 0) atomicOr(err, kErrIndex);
+      const bool want = i < hi_r && !(c & kForced);
+      const int64_t row = want && node < lr.nrows ? row_at<kPaged>(a, lr, node) : -1;
+      rs.ok[r] = row >= 0;
+      if (want && row < 0 && j16 == 0) atomicOr(err, kErrIndex);
       if (rs.ok[r]) {
-        rs.k[r] = ldg_row8(lr.k + node * kD, j16);
+        rs.k[r] = ldg_row8(lr.k + row * kD, j16);
         rs.tr[r] = ldg_trig4(a.table, i, j16);
-        if (values) rs.v[r] = ldg_row8(lr.v + node * kD, j16);
+        if (values) rs.v[r] = ldg_row8(lr.v + row * kD, j16);
       }
     }
   };
@@ -700,7 +724,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const Attend
     uint32_t *sk = skey_all + ((CS > 1) ? (lvl & 1) * MC : 0);
     float *slog = slog_all + (lvl & 1) * G * OWN;
     const bool single = hi_r - lo_r <= PASS;
-    const LevelRows lr = level_rows(a, geo, lvl, t.bh);
+    const LevelRows lr = level_rows<kPaged>(a, geo, lvl, t.bh);
 
     const int nforced = (a.causal && n > 0 && (cl[n - 1] & kForced)) ? 1 : 0;
     const int m = n - nforced;
@@ -825,7 +849,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const Attend
       if (sel)
         for (int u = nkept + tid; u < a.top_k; u += kCtaThreads) sel[u] = -1;
       uint32_t *nx = cand + (cur ^ 1) * MC;
-      const LevelRows lb = level_rows(a, geo, lvl - 1, t.bh);
+      const LevelRows lb = level_rows<kPaged>(a, geo, lvl - 1, t.bh);
       auto expand_one = [&](uint32_t v, int e) {  // children of the e-th expanded node
         bool lf = false;
         const int nch = child_count(a, geo, v, lvl, t.p, &lf);
@@ -835,7 +859,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const Attend
           nx[off + u] = (uint32_t)(first + u) | ((lf && u == nch - 1) ? kForced : 0u);
         if (off + nch > MC) atomicOr(err, kErrCount);
         atomicMax(next_count, min(off + nch, MC));
-        if (nch > 0 && e % CS == crank && first + nch <= lb.nrows) {
+        if (nch > 0 && e % CS == crank && first + nch <= lb.nrows && !(kPaged && lb.pages)) {
           prefetch_l2(lb.k + (int64_t)first * kD, (uint32_t)nch * kRowBytes);
           prefetch_l2(lb.v + (int64_t)first * kD, (uint32_t)nch * kRowBytes);
         }
@@ -894,7 +918,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const Attend
       //    are in node order and all but the last have exactly b children, so the e-th
       //    expanded candidate's children start at position e * b.
       uint32_t *nx = cand + (cur ^ 1) * MC;
-      const LevelRows lb = level_rows(a, geo, lvl - 1, t.bh);
+      const LevelRows lb = level_rows<kPaged>(a, geo, lvl - 1, t.bh);
       int carry_e = 0, carry_k = 0;
       int32_t *sel = (a.sel_idx != nullptr && crank == 0 && lvl <= a.sel_levels)
                          ? a.sel_idx + ((int64_t)tile * a.sel_levels + (lvl - 1)) * a.top_k
@@ -986,9 +1010,10 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const Attend
           rs.pos[r] = i;
           const uint32_t c = i < hi_r ? cl[i] : (kForced | kKept);
           const int64_t node = c & kNodeMask;
-          ent[r] = i < hi_r && !(c & (kForced | kKept)) && node < lr.nrows;
+          const int64_t row = i < hi_r && !(c & (kForced | kKept)) && node < lr.nrows ? row_at<kPaged>(a, lr, node) : -1;
+          ent[r] = row >= 0;
           rs.ok[r] = ent[r];
-          if (ent[r]) rs.v[r] = ldg_row8(lr.v + node * kD, j16);
+          if (ent[r]) rs.v[r] = ldg_row8(lr.v + row * kD, j16);
         }
         fold(rs, ent, slog, lo_r);
       }
@@ -1202,7 +1227,7 @@ __device__ __forceinline__ void rotated_query_regs(const uint2 (&qlo)[G], const 
 
 // Every slice of a level fits in RPH rows per half-warp: ceil(max_cand / CS) <= 16 RPH,
 // and max_cand <= kLeanMaxCand (the launcher checks both).
-template <int G, int CS, int RPH>
+template <int G, int CS, int RPH, bool kPaged = false>
 __global__ void __launch_bounds__(kCtaThreads, 1) attend_lean_kernel(const AttendArgs a) {
   static_assert(CS == 2 || CS == 4, "the lean kernel runs in clusters of 2 or 4");
   constexpr unsigned F = 0xffffffffu;
@@ -1254,11 +1279,12 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_lean_kernel(const Atten
   Trig4 ctr[RPH], ntr[RPH];
   bool cok[RPH], nok[RPH];
   auto load_row = [&](const LevelRows &lr, int pos, int node, bool valid, Row8 &k, Row8 &v, Trig4 &tr, bool &ok) {
-    ok = valid && node >= 0 && node < lr.nrows;
+    const int64_t row = valid && node >= 0 && node < lr.nrows ? row_at<kPaged>(a, lr, node) : -1;
+    ok = row >= 0;
     if (valid && !ok && j16 == 0) atomicOr(err, kErrIndex);
     if (ok) {
-      k = ld_row8_now(lr.k + (int64_t)node * kD, j16);
-      v = ld_row8_now(lr.v + (int64_t)node * kD, j16);
+      k = ld_row8_now(lr.k + row * kD, j16);
+      v = ld_row8_now(lr.v + row * kD, j16);
       tr = ld_trig4_now(a.table, pos, j16);
     }
   };
@@ -1273,7 +1299,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_lean_kernel(const Atten
   int per = (n + CS - 1) / CS;
   int lo = min(n, crank * per), hi = min(n, lo + per);
   {
-    const LevelRows lr = level_rows(a, geo, t.T, t.bh);
+    const LevelRows lr = level_rows<kPaged>(a, geo, t.T, t.bh);
 #pragma unroll
     for (int r = 0; r < RPH; ++r) {
       const int pos = lo + hw + kHalfWarps * r;
@@ -1382,7 +1408,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_lean_kernel(const Atten
     }
     // the ranking reads whole chunks of 8: positions n .. n rounded up to 8 score nothing
     if (tid < 8 && n + tid < ((n + 7) & ~7)) kbuf[pb * kLeanMaxCand + n + tid] = 0u;
-    const LevelRows lb = level_rows(a, geo, lvl - 1, t.bh);
+    const LevelRows lb = level_rows<kPaged>(a, geo, lvl - 1, t.bh);
     cluster_barrier();
 
     // 3. rank: candidate c is kept when fewer than top_k scorable candidates beat it
@@ -1593,7 +1619,7 @@ __host__ __device__ inline int warp_slice_bytes(int G, int max_cand) {
   return (G * kD + (4 + G) * max_cand) * 4;  // q, 2 candidate lists, logits, keys, entry list
 }
 
-template <int G>
+template <int G, bool kPaged = false>
 __global__ void __launch_bounds__(kWarpKernelMaxWarps * 32, (G <= 4 ? 2 : 1)) attend_warp_kernel(const AttendArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
@@ -1648,7 +1674,7 @@ __global__ void __launch_bounds__(kWarpKernelMaxWarps * 32, (G <= 4 ? 2 : 1)) at
         if (lane == 0) atomicOr(err, kErrCount);
         n = a.table_rows_needed - 1;
       }
-      const LevelRows lr = level_rows(a, geo, lvl, t.bh);
+      const LevelRows lr = level_rows<kPaged>(a, geo, lvl, t.bh);
       float2 q2lo[G][2], q2hi[G][2];
       {
         float qlo[G][4], qhi[G][4];
@@ -1663,10 +1689,11 @@ __global__ void __launch_bounds__(kWarpKernelMaxWarps * 32, (G <= 4 ? 2 : 1)) at
       auto fetch = [&](int i) {
         const uint32_t c = i < n ? cl[i] : kForced;
         const int64_t node = c & kNodeMask;
-        ok_n = i < n && !(c & kForced) && node < lr.nrows;
-        if (i < n && !(c & kForced) && node >= lr.nrows && j16 == 0) atomicOr(err, kErrIndex);
+        const int64_t row = i < n && !(c & kForced) && node < lr.nrows ? row_at<kPaged>(a, lr, node) : -1;
+        ok_n = row >= 0;
+        if (i < n && !(c & kForced) && row < 0 && j16 == 0) atomicOr(err, kErrIndex);
         if (ok_n) {
-          kr_n = ldg_row8(lr.k + node * kD, j16);
+          kr_n = ldg_row8(lr.k + row * kD, j16);
           tr_n = ldg_trig4(a.table, i, j16);
         }
       };
@@ -1753,8 +1780,8 @@ __global__ void __launch_bounds__(kWarpKernelMaxWarps * 32, (G <= 4 ? 2 : 1)) at
 #pragma unroll
         for (int u = 0; u < 8; ++u)
           if (e0 + u < ne) {
-            const int64_t node = cl[list[e0 + u]] & kNodeMask;
-            vv[u] = __ldg(reinterpret_cast<const uint2 *>(lr.v + node * kD + 4 * lane));
+            const int64_t row = row_at<kPaged>(a, lr, cl[list[e0 + u]] & kNodeMask);  // < 0: flagged by the key pass
+            vv[u] = row >= 0 ? __ldg(reinterpret_cast<const uint2 *>(lr.v + row * kD + 4 * lane)) : make_uint2(0u, 0u);
           }
 #pragma unroll
         for (int u = 0; u < 8; ++u)
@@ -1820,7 +1847,7 @@ int sm_count_cached() {
   return n > 0 ? n : 148;
 }
 
-template <int G, int CS>
+template <int G, int CS, bool kPaged>
 int launch_cta(const AttendArgs &args, cudaStream_t stream) {
   AttendArgs a = args;
   a.own_max = ((a.max_cand + CS - 1) / CS + 31) / 32 * 32;
@@ -1829,7 +1856,7 @@ int launch_cta(const AttendArgs &args, cudaStream_t stream) {
     set_error("attend needs %d bytes of shared memory per CTA (limit 232448)", L.total);
     return -1;
   }
-  auto kern = attend_cta_kernel<G, CS>;
+  auto kern = attend_cta_kernel<G, CS, kPaged>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
   if (e != cudaSuccess) return (int)e;
   if constexpr (CS == 1) {
@@ -1854,7 +1881,7 @@ int launch_cta(const AttendArgs &args, cudaStream_t stream) {
   }
 }
 
-template <int G>
+template <int G, bool kPaged>
 int launch_warp(const AttendArgs &args, cudaStream_t stream) {
   AttendArgs a = args;
   const int slice = warp_slice_bytes(G, a.max_cand);
@@ -1868,7 +1895,7 @@ int launch_warp(const AttendArgs &args, cudaStream_t stream) {
   }
   a.warps_per_block = wpb;
   const int smem = wpb * slice + kGeoBytes;
-  auto kern = attend_warp_kernel<G>;
+  auto kern = attend_warp_kernel<G, kPaged>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return (int)e;
   int per_sm = 0;
@@ -1881,10 +1908,10 @@ int launch_warp(const AttendArgs &args, cudaStream_t stream) {
   return (int)cudaGetLastError();
 }
 
-template <int G, int CS, int RPH>
+template <int G, int CS, int RPH, bool kPaged>
 int launch_lean_shape(const AttendArgs &a, cudaStream_t stream) {
   const LeanLayout L = lean_layout(G, CS, a.max_cand);
-  auto kern = attend_lean_kernel<G, CS, RPH>;
+  auto kern = attend_lean_kernel<G, CS, RPH, kPaged>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
   if (e != cudaSuccess) return (int)e;
   cudaLaunchConfig_t cfg = {};
@@ -1906,31 +1933,38 @@ int launch_lean_shape(const AttendArgs &a, cudaStream_t stream) {
 
 // The lean cluster kernel where its slices fit in registers; kNoLeanShape otherwise.
 constexpr int kNoLeanShape = -3;
-template <int G>
+template <int G, bool kPaged>
 int launch_lean(const AttendArgs &a, int CS, cudaStream_t stream) {
   const int mc = a.max_cand;
   if (mc > kLeanMaxCand) return kNoLeanShape;
-  if (CS == 4 && mc <= 4 * kHalfWarps * 2) return launch_lean_shape<G, 4, 2>(a, stream);
+  if (CS == 4 && mc <= 4 * kHalfWarps * 2) return launch_lean_shape<G, 4, 2, kPaged>(a, stream);
   if constexpr (G <= 4) {
-    if (CS == 4 && mc <= 4 * kHalfWarps * 3) return launch_lean_shape<G, 4, 3>(a, stream);
-    if (CS == 2 && mc <= 2 * kHalfWarps * 4) return launch_lean_shape<G, 2, 4>(a, stream);
+    if (CS == 4 && mc <= 4 * kHalfWarps * 3) return launch_lean_shape<G, 4, 3, kPaged>(a, stream);
+    if (CS == 2 && mc <= 2 * kHalfWarps * 4) return launch_lean_shape<G, 2, 4, kPaged>(a, stream);
   }
   return kNoLeanShape;
 }
 
-template <int G>
-int launch_g(const AttendArgs &a, int kernel, int CS, cudaStream_t stream) {
-  if (kernel == 2) return launch_warp<G>(a, stream);
+// kPaged: the token caches are a paged pool (level-0 rows through the page table); the
+// contiguous kernels carry no trace of it.
+template <int G, bool kPaged>
+int launch_gp(const AttendArgs &a, int kernel, int CS, cudaStream_t stream) {
+  if (kernel == 2) return launch_warp<G, kPaged>(a, stream);
   if (kernel == 3) {
-    const int rc = launch_lean<G>(a, CS, stream);
+    const int rc = launch_lean<G, kPaged>(a, CS, stream);
     if (rc != kNoLeanShape) return rc;
   }
   switch (CS) {
-    case 1: return launch_cta<G, 1>(a, stream);
-    case 2: return launch_cta<G, 2>(a, stream);
-    case 4: return launch_cta<G, 4>(a, stream);
+    case 1: return launch_cta<G, 1, kPaged>(a, stream);
+    case 2: return launch_cta<G, 2, kPaged>(a, stream);
+    case 4: return launch_cta<G, 4, kPaged>(a, stream);
     default: return -2;
   }
+}
+
+template <int G>
+int launch_g(const AttendArgs &a, int kernel, int CS, cudaStream_t stream) {
+  return a.page_table ? launch_gp<G, true>(a, kernel, CS, stream) : launch_gp<G, false>(a, kernel, CS, stream);
 }
 
 }  // namespace
@@ -1958,6 +1992,9 @@ int launch_attend(const AttendLaunch &l, void *stream) {
   a.cap = l.geom.capacity;
   a.length = l.length;
   a.seq_len = l.tree.seq_len;
+  a.page_table = l.tree.page_table;
+  a.page_shift = l.tree.page_table ? __builtin_ctz((unsigned)l.tree.page_size) : 0;
+  a.num_pages = l.tree.page_table ? l.tree.num_pages : 0;
   for (int i = 0; i <= kMaxLevels; ++i) {
     a.row_off[i] = l.geom.row_off[i];
     a.slots[i] = l.geom.slots[i];

@@ -45,7 +45,29 @@ struct BuildArgs {
   int32_t hkv;
   int64_t span;           // tokens under a level l node (b^l)
   const int64_t *seq_len; // per-sequence lengths (NULL: every sequence has `length`)
+  const int32_t *pages;   // level 1 over a paged token cache: the page table (else NULL)
+  int64_t pages_per_seq;
+  int32_t page_shift, num_pages;
   const float *pooler;    // [128][128] row-major W
+};
+
+// Rows of one (sequence, head) of the level below, relative to its base: contiguous...
+struct PlainRows {
+  static constexpr bool kPaged = false;
+  __device__ __forceinline__ int64_t operator()(int64_t c) const { return c; }
+};
+// ...or token rows of a paged cache, base = head h's rows of page 0 (pages are
+// Hkv * page_size rows apart); -1 for a page outside the pool (the row is skipped).
+struct PagedRows {
+  static constexpr bool kPaged = true;
+  const int32_t *pages;  // this sequence's page table
+  int64_t stride;        // Hkv << shift
+  int shift, num_pages;
+  __device__ __forceinline__ int64_t operator()(int64_t c) const {
+    const int pg = __ldg(pages + (c >> shift));
+    if ((unsigned)pg >= (unsigned)num_pages) return -1;
+    return (int64_t)pg * stride + (c & ((int64_t(1) << shift) - 1));
+  }
 };
 
 // Wt[k][o] = W[o][k] into shared memory.  A thread moves 16-byte pieces of W; the 32 lanes of
@@ -87,16 +109,18 @@ __device__ __forceinline__ uint2 ld_child(const uint16_t *p) {
 // stored keys.  Value: token-count-weighted mean; every child but the level's last covers
 // span_prev tokens, so the children are summed with weight 1 and the last child, if it covers
 // fewer tokens, then gets its share f = tokens / span_prev.
-template <bool kReadOnly>
+template <bool kReadOnly, class Rows>
 __device__ __forceinline__ void node_means(const uint16_t *kb, const uint16_t *vb, int64_t c0, int64_t c1,
                                            int64_t n_prev, int64_t length, int64_t span_prev, float ks[4],
-                                           float vs[4]) {
+                                           float vs[4], const Rows &rows) {
   float2 ks2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // dims (0,1), (2,3) of the lane's 4
   float2 vs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll 16  // a whole node's children (b = 16) in flight at once
   for (int64_t c = c0; c < c1; ++c) {
-    const uint2 ku = ld_child<kReadOnly>(kb + c * kD);
-    const uint2 vu = ld_child<kReadOnly>(vb + c * kD);
+    const int64_t r = rows(c);
+    if (Rows::kPaged && r < 0) continue;
+    const uint2 ku = ld_child<kReadOnly>(kb + r * kD);
+    const uint2 vu = ld_child<kReadOnly>(vb + r * kD);
     ks2[0] = __fadd2_rn(ks2[0], make_float2(bf16_lo(ku.x), bf16_hi(ku.x)));
     ks2[1] = __fadd2_rn(ks2[1], make_float2(bf16_lo(ku.y), bf16_hi(ku.y)));
     vs2[0] = __fadd2_rn(vs2[0], make_float2(bf16_lo(vu.x), bf16_hi(vu.x)));
@@ -110,7 +134,8 @@ __device__ __forceinline__ void node_means(const uint16_t *kb, const uint16_t *v
     const int64_t last_tokens = length - (c1 - 1) * span_prev;
     if (last_tokens < span_prev) {
       const float f1 = (float)last_tokens / (float)span_prev - 1.f;
-      const uint2 vu = ld_child<kReadOnly>(vb + (c1 - 1) * kD);
+      const int64_t r = rows(c1 - 1);
+      const uint2 vu = (Rows::kPaged && r < 0) ? make_uint2(0u, 0u) : ld_child<kReadOnly>(vb + r * kD);
       vs[0] = __fmaf_rn(f1, bf16_lo(vu.x), vs[0]);
       vs[1] = __fmaf_rn(f1, bf16_hi(vu.x), vs[1]);
       vs[2] = __fmaf_rn(f1, bf16_lo(vu.y), vs[2]);
@@ -176,7 +201,7 @@ __device__ __forceinline__ void store_row4(uint16_t *p, const float x[4]) {
 // (lane = 4 consecutive dims, one 256-byte row per warp load), forms the child means in
 // fp32, writes the value rows, then applies W to its own key means (W^T resident in shared
 // memory).  Warps share only W^T, so they never wait for one another after it is loaded.
-template <int NPW>
+template <int NPW, bool kPaged>
 __global__ void __launch_bounds__(kBuildThreads, 2) build_level_kernel(const BuildArgs a) {
   constexpr int kNodesPerBlock = kBuildWarps * NPW;
   extern __shared__ __align__(16) float smem_f[];
@@ -207,9 +232,18 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_level_kernel(const Bui
         if (live[t]) {
           const int64_t c0 = j * a.b;
           const int64_t c1 = min(c0 + (int64_t)a.b, n_prev);
-          const uint16_t *kb = a.src_k + (a.src_row_off + bhi * a.src_slots) * kD + lane * 4;
-          const uint16_t *vb = a.src_v + (a.src_row_off + bhi * a.src_slots) * kD + lane * 4;
-          node_means<true>(kb, vb, c0, c1, n_prev, length, a.span_prev, ks, vs);
+          if (kPaged) {  // level 1 over a paged token cache
+            const int64_t h = bhi % a.hkv;
+            const PagedRows rows{a.pages + (bhi / a.hkv) * a.pages_per_seq, (int64_t)a.hkv << a.page_shift,
+                                 a.page_shift, a.num_pages};
+            const uint16_t *kb = a.src_k + (h << a.page_shift) * kD + lane * 4;
+            const uint16_t *vb = a.src_v + (h << a.page_shift) * kD + lane * 4;
+            node_means<true>(kb, vb, c0, c1, n_prev, length, a.span_prev, ks, vs, rows);
+          } else {
+            const uint16_t *kb = a.src_k + (a.src_row_off + bhi * a.src_slots) * kD + lane * 4;
+            const uint16_t *vb = a.src_v + (a.src_row_off + bhi * a.src_slots) * kD + lane * 4;
+            node_means<true>(kb, vb, c0, c1, n_prev, length, a.span_prev, ks, vs, PlainRows{});
+          }
           store_row4(a.dst_v + (a.dst_row_off + bhi * a.dst_slots + j) * kD + lane * 4, vs);
         }
       }
@@ -249,6 +283,8 @@ struct ExtendArgs {
   uint16_t *k_node, *v_node;    // node arena
   const float *pooler;
   const int64_t *seq_len;       // per-sequence lengths before the append (NULL: all `at`)
+  const int32_t *pages;         // paged token cache: the page table (NULL: contiguous)
+  int32_t page_shift, num_pages;
   int64_t capacity;
   int64_t at;                   // first new slot (the length before the append; the longest one)
   int32_t chunk, hkv, b, levels;  // levels = T(at + chunk)
@@ -266,6 +302,7 @@ __device__ __forceinline__ void prefetch_l2(const void *p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
+template <bool kPaged>
 __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendArgs a) {
   extern __shared__ __align__(16) float smem_f[];
   float *Wt = smem_f;               // swizzled W^T (staging only)
@@ -287,6 +324,12 @@ __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendA
     *j0 = l <= t_old ? at / a.span[l] : 0;
     *j1 = (length + a.span[l] - 1) / a.span[l];
   };
+  // token t of this (sequence, head): row tok_base + tok_row(t), -1 for a page outside the pool
+  const int64_t h = bhi % a.hkv;
+  const int64_t tok_base = kPaged ? (h << a.page_shift) * kD : bhi * a.capacity * kD;
+  const PagedRows paged{kPaged ? a.pages + (bhi / a.hkv) * (a.capacity >> a.page_shift) : nullptr,
+                        (int64_t)a.hkv << a.page_shift, a.page_shift, a.num_pages};
+  auto tok_row = [&](int64_t t) -> int64_t { return kPaged ? paged(t) : t; };
 
   // W in flight (a warp reads one 512-byte row) while the tokens are appended and the first
   // children load
@@ -295,13 +338,14 @@ __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendA
 #pragma unroll
   for (int i = 0; i < kPieces; ++i) w[i] = __ldg(reinterpret_cast<const float4 *>(a.pooler) + tid + i * kExtendThreads);
   {
-    const int64_t s = bhi / a.hkv, h = bhi % a.hkv;
-    uint4 *kt = reinterpret_cast<uint4 *>(a.k_tok + (bhi * a.capacity + at) * kD);
-    uint4 *vt = reinterpret_cast<uint4 *>(a.v_tok + (bhi * a.capacity + at) * kD);
+    const int64_t s = bhi / a.hkv;
     for (int e = tid; e < a.chunk * 16; e += kExtendThreads) {  // 16 pieces a row
       const int64_t src = ((s * a.chunk + (e >> 4)) * a.hkv + h) * 16 + (e & 15);
-      kt[e] = __ldg(a.k_new + src);
-      vt[e] = __ldg(a.v_new + src);
+      const int64_t row = tok_row(at + (e >> 4));
+      if (row < 0) continue;
+      const int64_t dst = (tok_base + row * kD) / 8 + (e & 15);  // in 16-byte pieces
+      reinterpret_cast<uint4 *>(a.k_tok)[dst] = __ldg(a.k_new + src);
+      reinterpret_cast<uint4 *>(a.v_tok)[dst] = __ldg(a.v_new + src);
     }
   }
   // every child row the walk reads above level 1, into L2 ahead of the dependent levels
@@ -325,15 +369,20 @@ __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendA
     const int64_t n_prev = (length + span_prev - 1) / span_prev;
     int64_t j0, j1;
     node_range(l, &j0, &j1);
-    const uint16_t *src = l == 1 ? (is_v ? a.v_tok : a.k_tok) + bhi * a.capacity * kD
+    const uint16_t *src = l == 1 ? (is_v ? a.v_tok : a.k_tok) + tok_base
                                  : (is_v ? a.v_node : a.k_node) + (a.row_off[l - 1] + bhi * a.slots[l - 1]) * kD;
     uint16_t *dk = a.k_node + (a.row_off[l] + bhi * a.slots[l]) * kD;
     uint16_t *dv = a.v_node + (a.row_off[l] + bhi * a.slots[l]) * kD;
     for (int64_t j = j0; j < j1; ++j) {
       const int64_t c0 = j * a.b, c1 = min(c0 + (int64_t)a.b, n_prev);
+      // the level below's row of child c (tokens through the page table when paged)
+      auto child = [&](int64_t c) -> int64_t { return l == 1 ? tok_row(c) : c; };
       float sum = 0.f;
 #pragma unroll 16
-      for (int64_t c = c0; c < c1; ++c) sum += bf16_lo(src[c * kD + d]);
+      for (int64_t c = c0; c < c1; ++c) {
+        const int64_t r = child(c);
+        if (r >= 0) sum += bf16_lo(src[r * kD + d]);
+      }
       const float nch = (float)(c1 - c0);
       if (is_v) {  // token-weighted: the level's last child gets its share tokens / span_prev
         float wsum = nch;
@@ -341,7 +390,8 @@ __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendA
           const int64_t last_tokens = length - (c1 - 1) * span_prev;
           if (last_tokens < span_prev) {
             const float f1 = (float)last_tokens / (float)span_prev - 1.f;
-            sum = __fmaf_rn(f1, bf16_lo(src[(c1 - 1) * kD + d]), sum);
+            const int64_t r = child(c1 - 1);
+            sum = __fmaf_rn(f1, r >= 0 ? bf16_lo(src[r * kD + d]) : 0.f, sum);
             wsum += f1;
           }
         }
@@ -400,8 +450,11 @@ __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendA
 }
 
 // k_new / v_new [B][C][Hkv][128] -> token caches [B][Hkv][capacity][128] at slot `at + i`.
+// With a page table the slot is row (at + i) % page_size of head h in page
+// pages[b][(at + i) / page_size]; a page outside the pool is skipped.
 __global__ void append_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new, uint16_t *k_tok,
-                              uint16_t *v_tok, int64_t capacity, int64_t at, int chunk, int hkv, int64_t rows) {
+                              uint16_t *v_tok, int64_t capacity, int64_t at, int chunk, int hkv, int64_t rows,
+                              const int32_t *pages, int page_shift, int num_pages) {
   const int64_t n16 = rows * 16;  // 16-byte pieces
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n16; e += (int64_t)gridDim.x * blockDim.x) {
     const int64_t row = e >> 4;
@@ -410,7 +463,15 @@ __global__ void append_kernel(const uint4 *__restrict__ k_new, const uint4 *__re
     const int64_t bi_i = row / hkv;
     const int64_t i = bi_i % chunk;
     const int64_t bi = bi_i / chunk;
-    const int64_t dst = ((bi * hkv + h) * capacity + at + i) * kD + part * 8;
+    int64_t dst;
+    if (pages) {
+      const int64_t t = at + i;
+      const int pg = __ldg(pages + bi * (capacity >> page_shift) + (t >> page_shift));
+      if ((unsigned)pg >= (unsigned)num_pages) continue;
+      dst = ((((int64_t)pg * hkv + h) << page_shift) + (t & ((int64_t(1) << page_shift) - 1))) * kD + part * 8;
+    } else {
+      dst = ((bi * hkv + h) * capacity + at + i) * kD + part * 8;
+    }
     reinterpret_cast<uint4 *>(k_tok + dst)[0] = k_new[e];
     reinterpret_cast<uint4 *>(v_tok + dst)[0] = v_new[e];
   }
@@ -454,13 +515,21 @@ int configure_smem() {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return (int)e;
   if (configured_device == dev) return 0;
-  e = cudaFuncSetAttribute(build_level_kernel<kNodesPerWarp>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(build_level_kernel<kNodesPerWarp, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)build_smem(kNodesPerWarp));
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(build_level_kernel<kFewNodes>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(build_level_kernel<kFewNodes, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)build_smem(kFewNodes));
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(extend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kExtendSmem);
+    e = cudaFuncSetAttribute(build_level_kernel<kNodesPerWarp, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)build_smem(kNodesPerWarp));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(build_level_kernel<kFewNodes, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)build_smem(kFewNodes));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(extend_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kExtendSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(extend_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kExtendSmem);
   if (e != cudaSuccess) return (int)e;
   configured_device = dev;
   return 0;
@@ -501,19 +570,24 @@ int launch_build_level(const TreeGeom &g, const recsa_tree &t, int level, int64_
   a.hkv = g.hkv;
   a.span = g.span[level];
   a.seq_len = t.seq_len;
+  a.pages = from_tokens ? t.page_table : nullptr;
+  a.page_shift = t.page_table ? __builtin_ctz((unsigned)t.page_size) : 0;
+  a.pages_per_seq = t.page_table ? g.capacity >> a.page_shift : 0;
+  a.num_pages = t.page_table ? t.num_pages : 0;
   a.pooler = t.pooler;
   const int rc = configure_smem();
   if (rc != 0) return rc;
   const int64_t nodes = (int64_t)a.bh * a.nj;
   const int64_t full_grid = (int64_t)sm_count() * 2;
-  if (nodes <= full_grid * kBuildWarps * kFewNodes) {  // fits one pass of warps with a node each
-    const int64_t grid = ceil_div(nodes, kBuildWarps * kFewNodes);
-    build_level_kernel<kFewNodes><<<(unsigned)grid, kBuildThreads, build_smem(kFewNodes), (cudaStream_t)stream>>>(a);
-  } else {
-    const int64_t grid = std::min<int64_t>(ceil_div(nodes, kBuildWarps * kNodesPerWarp), full_grid);
-    build_level_kernel<kNodesPerWarp>
-        <<<(unsigned)grid, kBuildThreads, build_smem(kNodesPerWarp), (cudaStream_t)stream>>>(a);
-  }
+  // one pass of warps with a node each when it fits, else 8 nodes a warp over a grid of 2 CTAs
+  // per SM; the paged instances read level 1 through the page table
+  const bool few = nodes <= full_grid * kBuildWarps * kFewNodes;
+  const int npw = few ? kFewNodes : kNodesPerWarp;
+  const int64_t grid = few ? ceil_div(nodes, kBuildWarps * kFewNodes)
+                           : std::min<int64_t>(ceil_div(nodes, kBuildWarps * kNodesPerWarp), full_grid);
+  auto kern = few ? (a.pages ? build_level_kernel<kFewNodes, true> : build_level_kernel<kFewNodes, false>)
+                  : (a.pages ? build_level_kernel<kNodesPerWarp, true> : build_level_kernel<kNodesPerWarp, false>);
+  kern<<<(unsigned)grid, kBuildThreads, build_smem(npw), (cudaStream_t)stream>>>(a);
   return (int)cudaGetLastError();
 }
 
@@ -528,6 +602,9 @@ int launch_extend(const TreeGeom &g, const recsa_tree &t, const void *k_new, con
   a.v_node = reinterpret_cast<uint16_t *>(t.v_node);
   a.pooler = t.pooler;
   a.seq_len = t.seq_len;
+  a.pages = t.page_table;
+  a.page_shift = t.page_table ? __builtin_ctz((unsigned)t.page_size) : 0;
+  a.num_pages = t.page_table ? t.num_pages : 0;
   a.capacity = g.capacity;
   a.at = at;
   a.chunk = chunk;
@@ -542,7 +619,8 @@ int launch_extend(const TreeGeom &g, const recsa_tree &t, const void *k_new, con
   const int rc = configure_smem();
   if (rc != 0) return rc;
   const int64_t grid = (int64_t)g.batch * g.hkv;
-  extend_kernel<<<(unsigned)grid, kExtendThreads, kExtendSmem, (cudaStream_t)stream>>>(a);
+  auto kern = a.pages ? extend_kernel<true> : extend_kernel<false>;
+  kern<<<(unsigned)grid, kExtendThreads, kExtendSmem, (cudaStream_t)stream>>>(a);
   return (int)cudaGetLastError();
 }
 
@@ -566,7 +644,7 @@ int launch_append(const TreeGeom &g, const recsa_tree &t, const void *k_new, con
   append_kernel<<<(unsigned)grid, threads, 0, (cudaStream_t)stream>>>(
       reinterpret_cast<const uint4 *>(k_new), reinterpret_cast<const uint4 *>(v_new),
       reinterpret_cast<uint16_t *>(t.k_tok), reinterpret_cast<uint16_t *>(t.v_tok), g.capacity, at, chunk, g.hkv,
-      rows);
+      rows, t.page_table, t.page_table ? __builtin_ctz((unsigned)t.page_size) : 0, t.page_table ? t.num_pages : 0);
   return (int)cudaGetLastError();
 }
 

@@ -107,7 +107,19 @@ typedef struct recsa_params {
  *                  after their kernels) as they advance `length` on the host.  The
  *                  kernels clamp an entry outside [0, length] into it; decode and prefill
  *                  calls also flag one in the workspace error word
- *                  (RECSA_ERR_DEVICE_CHECK from recsa_check_device_errors). */
+ *                  (RECSA_ERR_DEVICE_CHECK from recsa_check_device_errors).
+ *   page_table   : NULL for the contiguous caches above.  Otherwise the token caches are
+ *                  a paged pool: k_tok, v_tok are bf16 [num_pages][Hkv][page_size][128],
+ *                  and page_table is a device array int32 [batch][capacity / page_size],
+ *                  4-byte aligned, owned by the caller: token t of sequence s sits in
+ *                  page page_table[s][t / page_size], row t % page_size.  page_size is a
+ *                  power of two (1 .. 65536) dividing capacity; num_pages >= 1.  Every
+ *                  call reads the same rows as with contiguous caches (the results are
+ *                  identical); appends write into the pages the table names, so the
+ *                  caller maps a sequence's pages before its tokens reach them.  A table
+ *                  entry outside [0, num_pages) is never dereferenced: the attend kernels
+ *                  skip the row and flag it (RECSA_ERR_DEVICE_CHECK), the build and append
+ *                  kernels skip it (such a tree holds undefined rows). */
 typedef struct recsa_tree {
   int32_t batch;
   int32_t reserved;
@@ -119,6 +131,9 @@ typedef struct recsa_tree {
   void *v_node;
   const float *pooler;
   int64_t *seq_len;
+  const int32_t *page_table;
+  int32_t page_size;
+  int32_t num_pages;
 } recsa_tree;
 
 /* Optional diagnostics and launch-shape overrides of recsa_decode / recsa_prefill_chunk

@@ -180,6 +180,21 @@ def test_append_capacity_and_arguments_rejected():
     assert t.length == 4000  # unchanged on failure
 
 
+@pytest.mark.parametrize("kw", [
+    dict(page_size=3),                     # not a power of two
+    dict(page_size=0),
+    dict(page_size=1 << 17),               # above 65536
+    dict(page_size=8, capacity=4100),      # capacity not a multiple of the page size
+    dict(page_size=8, num_pages=0),
+    dict(page_size=8, page_table=FAKE + 2),  # misaligned table
+])
+def test_paged_cache_arguments_rejected(kw):
+    p = _p()
+    d = dict(length=100, page_table=FAKE, page_size=8, num_pages=16)
+    d.update(kw)
+    assert lib.recsa_build_tree(ctypes.byref(p), ctypes.byref(_tree(**d)), None) == INVALID
+
+
 def test_layout_and_build_reject_bad_input():
     p = _p()
     rows = ctypes.c_int64()
