@@ -298,6 +298,15 @@ constexpr int kHalfK = kD / 2;          // W columns held by each thread of a di
 // and the per-thread row reads both hit 32 distinct banks.
 constexpr size_t kExtendSmem = (size_t)(kD * kD + 2 * kD) * sizeof(float);
 
+// x / y and ceil(x / y) for x >= 0, y >= 1, in 32 bits whenever the operands fit (a 64-bit
+// division is a long instruction sequence; lengths and spans of real trees fit 32 bits).
+__device__ __forceinline__ int64_t div_nn(int64_t x, int64_t y) {
+  if (y > x) return 0;
+  if (x <= 0xffffffffLL) return (int64_t)((uint32_t)x / (uint32_t)y);
+  return x / y;
+}
+__device__ __forceinline__ int64_t ceil_div_nn(int64_t x, int64_t y) { return x > 0 ? div_nn(x - 1, y) + 1 : 0; }
+
 __device__ __forceinline__ void prefetch_l2(const void *p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
@@ -321,8 +330,8 @@ __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendA
   // level l rebuilds nodes [j0, j1): those whose spans meet the new tokens (a level that
   // becomes new is built whole)
   auto node_range = [&](int l, int64_t *j0, int64_t *j1) {
-    *j0 = l <= t_old ? at / a.span[l] : 0;
-    *j1 = (length + a.span[l] - 1) / a.span[l];
+    *j0 = l <= t_old ? div_nn(at, a.span[l]) : 0;
+    *j1 = ceil_div_nn(length, a.span[l]);
   };
   // token t of this (sequence, head): row tok_base + tok_row(t), -1 for a page outside the pool
   const int64_t h = bhi % a.hkv;
@@ -351,7 +360,7 @@ __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendA
   // every child row the walk reads above level 1, into L2 ahead of the dependent levels
   // (K and V, two 128-byte lines each)
   for (int l = 2; l <= t_new; ++l) {
-    const int64_t n_prev = (length + a.span[l - 1] - 1) / a.span[l - 1];
+    const int64_t n_prev = ceil_div_nn(length, a.span[l - 1]);
     int64_t j0, j1;
     node_range(l, &j0, &j1);
     const int64_t c0 = j0 * a.b, c1 = min(j1 * a.b, n_prev);
@@ -366,7 +375,7 @@ __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendA
   const int kbase = is_v ? kHalfK : 0;
   for (int l = 1; l <= t_new; ++l) {
     const int64_t span_prev = a.span[l - 1];
-    const int64_t n_prev = (length + span_prev - 1) / span_prev;
+    const int64_t n_prev = ceil_div_nn(length, span_prev);
     int64_t j0, j1;
     node_range(l, &j0, &j1);
     const uint16_t *src = l == 1 ? (is_v ? a.v_tok : a.k_tok) + tok_base
