@@ -529,6 +529,24 @@ def run_profile_case(args):
             R.append(p, tree, kn, vn)
         torch.cuda.synchronize()
         print(json.dumps({"profile": "append", "length": tree.length, "kv_heads": w.kv_heads}))
+    elif args.profile == "decode_loop":
+        w = I.WORKLOADS["decode_1m"]
+        steps = 24
+        inp = I.decode_inputs(w, device="cuda", capacity=w.length + steps + 8)
+        p = R.params(num_kv_heads=w.kv_heads, num_q_heads=w.q_heads, branching=w.branching, top_k=w.top_k)
+        tree, ws = make_tree(R, p, inp, w.length)
+        g = torch.Generator(device="cuda").manual_seed(5)
+        B, Hkv, Hq = w.batch, w.kv_heads, w.q_heads
+        out = torch.empty(B, 1, Hq, 128, dtype=torch.bfloat16, device="cuda")
+        flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        for _ in range(steps):  # append + decode per step, L2 flushed before each as in the bench
+            kn, vn, qn = (torch.randn(B, 1, h, 128, generator=g, device="cuda").to(torch.bfloat16)
+                          for h in (Hkv, Hkv, Hq))
+            flush.zero_()
+            R.append(p, tree, kn, vn)
+            R.decode(p, tree, qn, out, ws)
+        R.check_device_errors(ws)
+        print(json.dumps({"profile": "decode_loop", "steps": steps, "length": tree.length}))
     elif args.profile == "build":
         w = dataclasses.replace(I.WORKLOADS["build_decode_2m"], length=1 << 19)
         inp = I.decode_inputs(w, device="cuda")
@@ -648,7 +666,7 @@ def main():
     ap.add_argument("--shard", default="sequences", choices=["sequences", "heads"],
                     help="with N GPUs: N replicas of the batch (sequences, weak scaling) or the batch's "
                          "KV heads split over the N GPUs (heads, strong scaling)")
-    ap.add_argument("--profile", choices=["decode", "prefill", "build", "append"], help="run a small case of one kernel for ncu")
+    ap.add_argument("--profile", choices=["decode", "prefill", "build", "append", "decode_loop"], help="run a small case of one kernel for ncu")
     args = ap.parse_args()
     if args.profile:
         run_profile_case(args)
