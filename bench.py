@@ -371,6 +371,41 @@ def leg_decode_varlen(R, timer, args, dist_on):
     return res
 
 
+def leg_decode_paged(R, timer, args, dist_on):
+    """The headline decode (1M, B = 4) over a paged token cache: pages of 64 tokens in a pool
+    placed by a shuffled page table, next to the same caches stored contiguously."""
+    w = I.WORKLOADS["decode_1m"]
+    inp = I.decode_inputs(w, device="cuda")
+    p = R.params(num_kv_heads=w.kv_heads, num_q_heads=w.q_heads, branching=w.branching, top_k=w.top_k)
+    P = 64
+    B, H, cap = w.batch, w.kv_heads, w.length
+    pps = cap // P
+    g = torch.Generator(device="cpu").manual_seed(17)
+    perm = torch.randperm(B * pps, generator=g).to(torch.int32)
+    table = perm.view(B, pps).contiguous().cuda()
+    pools = []
+    for x in (inp["k_tok"], inp["v_tok"]):
+        pool = torch.empty(B * pps, H, P, 128, dtype=torch.bfloat16, device="cuda")
+        pool[perm.long().cuda()] = x.view(B, H, pps, P, 128).permute(0, 2, 1, 3, 4).reshape(B * pps, H, P, 128)
+        pools.append(pool)
+    q = inp["q"]
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
+    steps = max(20, args.steps // 10) if not args.quick else 20
+    res = {"workload": f"decode_paged_1m: B={B}, L={w.length}, pages of {P} tokens, shuffled table, "
+                       f"Hq={w.q_heads}, Hkv={H}, b={w.branching}, k={w.top_k}, 1 query per sequence"}
+    del inp["k_tok"], inp["v_tok"]
+    tree = R.RecsaTree(p, pools[0], pools[1], inp["pooler"], w.length, page_table=table)
+    ws = R.Workspace(p, tree.capacity, "cuda")
+    R.build_tree(p, tree)
+    per, _ = timer.run(lambda: R.decode(p, tree, q, out, ws), steps, 3)
+    t = max_over_ranks(sum(per), dist_on) / steps
+    R.check_device_errors(ws)
+    res["paged"] = {"queries_per_s": B / t, "us_per_call": t * 1e6}
+    del tree, ws, pools, table
+    torch.cuda.empty_cache()
+    return res
+
+
 def leg_build_2m(R, timer, args, dist_on, hbm_peak):
     w = I.WORKLOADS["build_decode_2m"]
     inp = I.decode_inputs(w, device="cuda")
@@ -589,6 +624,7 @@ def run_gpu(args):
         extra["build_2m"] = leg_build_2m(R, timer, args, dist_on, hbm_peak)
         extra["decode_loop_1m"] = leg_decode_loop(R, timer, args, dist_on)
         extra["decode_varlen"] = leg_decode_varlen(R, timer, args, dist_on)
+        extra["decode_paged_1m"] = leg_decode_paged(R, timer, args, dist_on)
     clk = clocks.stop()
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

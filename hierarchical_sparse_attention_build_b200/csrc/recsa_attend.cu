@@ -134,6 +134,14 @@ __device__ __forceinline__ int nodes_at(int p, int span) {
   return (int)(((uint32_t)p + (uint32_t)span - 1u) / (uint32_t)span);  // p < 2^31, span <= 2^30 + 1
 }
 
+// A per-sequence length outside [0, length] (tile_info clamped it) sets the index bit; one
+// thread per tile, after the tile's work.
+__device__ __forceinline__ void flag_bad_length(const AttendArgs &a, int s) {
+  if (!a.seq_len) return;
+  const int64_t raw = a.seq_len[s];
+  if (raw < 0 || raw > a.length) atomicOr(&a.hdr->err, kErrIndex);
+}
+
 // Candidate count of the top level; *forced_pos = position of the forced partial node or -1.
 __device__ __forceinline__ int top_candidates(const AttendArgs &a, const Geo &geo, const TileInfo &t,
                                               int *forced_pos) {
@@ -1036,6 +1044,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const Attend
     cur ^= 1;
   }
 
+  if (crank == 0 && tid == 0) flag_bad_length(a, t.s);
   if (a.entries != nullptr && crank == 0 && tid == 0) {
     a.entries[2 * (int64_t)tile] = keys_read;
     a.entries[2 * (int64_t)tile + 1] = values_read;
@@ -1538,6 +1547,7 @@ __global__ void __launch_bounds__(kCtaThreads, 1) attend_lean_kernel(const Atten
     hi = hi2;
   }
 
+  if (crank == 0 && tid == 0) flag_bad_length(a, t.s);
   if (a.entries != nullptr && crank == 0 && tid == 0) {
     a.entries[2 * (int64_t)tile] = keys_read;
     a.entries[2 * (int64_t)tile + 1] = values_read;
@@ -1823,6 +1833,7 @@ __global__ void __launch_bounds__(kWarpKernelMaxWarps * 32, (G <= 4 ? 2 : 1)) at
       store_out4(a, out0 + h * kD + 4 * lane, acc[h][0].x * inv, acc[h][0].y * inv, acc[h][1].x * inv,
                  acc[h][1].y * inv);
     }
+    if (lane == 0) flag_bad_length(a, t.s);
     if (a.entries != nullptr && lane == 0) {
       a.entries[2 * (int64_t)tile] = keys_read;
       a.entries[2 * (int64_t)tile + 1] = values_read;
@@ -1832,13 +1843,6 @@ __global__ void __launch_bounds__(kWarpKernelMaxWarps * 32, (G <= 4 ? 2 : 1)) at
 }
 
 // ================================================================== launch
-
-// Flags per-sequence lengths outside [0, length] in the workspace error word (the attend
-// kernels clamp them into that range).
-__global__ void check_lengths_kernel(const int64_t *seq_len, int batch, int64_t length, WsHeader *hdr) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < batch && (seq_len[i] < 0 || seq_len[i] > length)) atomicOr(&hdr->err, kErrIndex);
-}
 
 int sm_count_cached() {
   int dev = 0, n = 148;
@@ -1970,13 +1974,6 @@ int launch_g(const AttendArgs &a, int kernel, int CS, cudaStream_t stream) {
 }  // namespace
 
 int launch_attend(const AttendLaunch &l, void *stream) {
-  if (l.tree.seq_len) {
-    const int threads = 128;
-    check_lengths_kernel<<<(l.geom.batch + threads - 1) / threads, threads, 0, (cudaStream_t)stream>>>(
-        l.tree.seq_len, l.geom.batch, l.length, reinterpret_cast<WsHeader *>(l.ws));
-    const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return (int)e;
-  }
   AttendArgs a = {};
   a.k_tok = reinterpret_cast<const uint16_t *>(l.tree.k_tok);
   a.v_tok = reinterpret_cast<const uint16_t *>(l.tree.v_tok);

@@ -171,10 +171,10 @@ def test_varlen_append_decode_loop():
                 assert np.array_equal(bits(a)[s, :, :counts[lvl]], bits(b)[s, :, :counts[lvl]]), (s, lvl)
 
 
-def test_varlen_prefill_chunk_matches_oracle():
+@pytest.mark.parametrize("C", [20, 200])  # 200: several nodes a level in the one-launch update
+def test_varlen_prefill_chunk_matches_oracle(C):
     lens = [300, 0, 77, 1000]
-    C = 20
-    c = VarCase(lens, 2, 4, 4, 2, seed=21, chunk=C)
+    c = VarCase(lens, 2, 4, 4, 2, seed=21 + C, chunk=C)
     R.build_tree(c.p, c.tree)
     kn, vn, q = (c.inp[x].cuda().contiguous() for x in ("k_new", "v_new", "q"))
     out = torch.empty(c.B, C, 8, 128, dtype=torch.float32, device="cuda")
