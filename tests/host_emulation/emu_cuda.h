@@ -1,4 +1,4 @@
-// Host versions of the CUDA features the lean attend kernel uses, for running its source on
+// Host versions of the CUDA features the lean attend and append kernels use, for running their source on
 // host threads (test infrastructure): one std::thread per CUDA thread; __syncthreads, the
 // cluster barrier, __syncwarp, shuffles, ballots and warp reductions are real rendezvous
 // of the threads that must take part, and a barrier that does not complete within 20 s
@@ -121,6 +121,7 @@ inline void TBarrier::wait_gen(long my, int line) {
 struct ThreadIdx { unsigned x; };
 #define threadIdx (ThreadIdx{(unsigned)emu::t_tid})
 #define blockIdx (ThreadIdx{(unsigned)emu::t_block})
+#define gridDim (ThreadIdx{0u})  // no emulated kernel strides over the grid (declared for the source to compile)
 
 #define __syncthreads() emu::g_cta_bar[emu::t_crank].wait(__LINE__)
 #define __syncwarp(...) emu::g_warp_bar[emu::t_crank * 8 + emu::t_tid / 32].wait(__LINE__)
@@ -162,6 +163,8 @@ inline uint32_t __umulhi(uint32_t a, uint32_t b) { return (uint32_t)(((uint64_t)
 inline float __expf(float x) { return std::exp(x); }
 inline float2 __fmul2_rn(float2 a, float2 b) { return {a.x * b.x, a.y * b.y}; }
 inline float2 __ffma2_rn(float2 a, float2 b, float2 c) { return {std::fma(a.x, b.x, c.x), std::fma(a.y, b.y, c.y)}; }
+inline float2 __fadd2_rn(float2 a, float2 b) { return {a.x + b.x, a.y + b.y}; }
+inline float __fmaf_rn(float a, float b, float c) { return std::fma(a, b, c); }
 template <typename T>
 inline T __ldg(const T *p) { return *p; }
 inline uint32_t atomicOr(uint32_t *p, uint32_t v) { return __atomic_fetch_or(p, v, __ATOMIC_SEQ_CST); }
