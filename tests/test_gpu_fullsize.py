@@ -119,3 +119,42 @@ def test_prefill_524k_chunk_8192():
                        out[0, i, h * G:(h + 1) * G], gpu_selection(sel, tile, top), ent[tile])
     stats.assert_ok()
     print("prefill_524k", stats)
+
+
+def test_decode_loop_1m_append_then_decode():
+    """The decode loop the benchmark times (1M tokens, B = 4): two steps of recsa_append (one
+    token per sequence) + recsa_decode of its query; the sampled trees after both appends and
+    the last step's tiles against the oracle over L + 2 tokens."""
+    w = I.WORKLOADS["decode_1m"]
+    S = 2
+    inp = I.decode_inputs(w, device="cuda", capacity=w.length + S + 2)
+    p = _params(w)
+    tree = R.RecsaTree(p, inp["k_tok"], inp["v_tok"], inp["pooler"], w.length)
+    ws = R.Workspace(p, tree.capacity, "cuda")
+    R.build_tree(p, tree)
+    B, Hkv, Hq, G = w.batch, w.kv_heads, w.q_heads, w.q_heads // w.kv_heads
+    g = torch.Generator(device="cuda").manual_seed(61)
+    steps = [tuple(torch.randn(B, 1, h, 128, generator=g, device="cuda").to(torch.bfloat16) for h in (Hkv, Hkv, Hq))
+             for _ in range(S)]
+    tiles = B * Hkv
+    for kn, vn, qn in steps:
+        R.append(p, tree, kn, vn)
+        out = torch.empty(B, 1, Hq, 128, dtype=torch.float32, device="cuda")
+        sel = torch.full((tiles, tree.levels, w.top_k), -7, dtype=torch.int32, device="cuda")
+        ent = torch.zeros(tiles, 2, dtype=torch.int32, device="cuda")
+        R.decode(p, tree, qn, out, ws, sel_idx=sel, sel_levels=tree.levels, entries=ent)
+        R.check_device_errors(ws)
+    assert tree.length == w.length + S
+    out, sel, ent = out.cpu().numpy(), sel.cpu().numpy(), ent.cpu().numpy()
+    qb = bits(steps[-1][2])
+    stats = Stats()
+    for s, h in ((0, 0), (3, 7)):
+        kx = np.stack([bits(kn[s, 0, h]) for kn, _, _ in steps])
+        vx = np.stack([bits(vn[s, 0, h]) for _, vn, _ in steps])
+        t = _oracle_tree(inp, s, h, w.length, w.branching, kx, vx)
+        _check_rows(tree, t, s, h)
+        tile = s * Hkv + h
+        check_tile(stats, O.bf16_bits_to_f64(qb[s, 0, h * G:(h + 1) * G]), t, w.length + S, w.top_k, False,
+                   out[s, 0, h * G:(h + 1) * G], gpu_selection(sel, tile, t.top), ent[tile])
+    stats.assert_ok()
+    print("decode_loop_1m", stats)
