@@ -169,3 +169,14 @@ def test_page_outside_the_pool_is_flagged():
             R.check_device_errors(x.ws)
     R.build_tree(x.p, x.g)  # skips the page's rows; nothing to flag without a workspace
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("G,b,P,kernel,cluster_size", [
+    (8, 16, 16, 3, 4), (1, 3, 4, 1, 1), (2, 16, 32, 2, 0), (8, 4, 8, 1, 4),
+])
+def test_paged_other_group_sizes_equal_contiguous(G, b, P, kernel, cluster_size):
+    x = Pair(2, 2, G, 900, b, 4, P, seed=G + b + P, queries=2)
+    x.build()
+    x.assert_same_trees()
+    a, c = x.decode_both(x.inp["q"], kernel, cluster_size)
+    assert torch.equal(a, c)

@@ -215,3 +215,14 @@ def test_out_of_range_length_is_flagged():
     c.seq_len[1] = 300
     R.decode(c.p, c.tree, c.inp["q"].cuda().contiguous(), out, c.ws)
     R.check_device_errors(c.ws)
+
+
+@pytest.mark.parametrize("G,b,k,kernel,cluster_size", [
+    (1, 3, 2, 0, 0), (2, 16, 8, 3, 2), (8, 16, 8, 3, 4), (8, 4, 2, 1, 2), (2, 3, 3, 2, 0),
+])
+def test_varlen_decode_other_group_sizes(G, b, k, kernel, cluster_size):
+    lens = [900, 0, 1, 333]
+    c = VarCase(lens, 2, G, b, k, seed=G * 10 + b)
+    R.build_tree(c.p, c.tree)
+    out, sel, ent = c.decode(c.inp["q"], kernel, cluster_size)
+    c.check_decode(c.inp["q"], out, sel, ent, lens)
