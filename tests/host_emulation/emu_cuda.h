@@ -58,7 +58,7 @@ struct TBarrier {
   void wait_gen(long my, int line);
 };
 
-extern thread_local int t_tid, t_block, t_crank, t_cs;
+extern thread_local int t_tid, t_block, t_crank, t_cs, t_grid;
 extern thread_local long t_cluster_gen;  // cluster-barrier generation this thread arrived at
 extern thread_local unsigned char *t_smem;
 extern std::vector<unsigned char *> g_cluster_smem;  // per cluster rank
@@ -121,7 +121,7 @@ inline void TBarrier::wait_gen(long my, int line) {
 struct ThreadIdx { unsigned x; };
 #define threadIdx (ThreadIdx{(unsigned)emu::t_tid})
 #define blockIdx (ThreadIdx{(unsigned)emu::t_block})
-#define gridDim (ThreadIdx{0u})  // no emulated kernel strides over the grid (declared for the source to compile)
+#define gridDim (ThreadIdx{(unsigned)emu::t_grid})
 
 #define __syncthreads() emu::g_cta_bar[emu::t_crank].wait(__LINE__)
 #define __syncwarp(...) emu::g_warp_bar[emu::t_crank * 8 + emu::t_tid / 32].wait(__LINE__)

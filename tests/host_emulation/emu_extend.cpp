@@ -1,8 +1,9 @@
-// Runs the append kernel (extend_kernel: one CTA of 256 threads per (sequence, KV head)) on host
-// threads, one std::thread per CUDA thread, over inputs read from a case directory, and writes
-// the caches and the node arena back there.  Test infrastructure: it checks the kernel's
-// barriers (every thread reaches each one), its memory accesses (AddressSanitizer) and its
-// results, without a GPU.
+// Runs the append kernel (extend_kernel: one CTA of 256 threads per (sequence, KV head)) or, with
+// "mode 1", every level of the tree build (build_level_kernel, one launch per level, a grid of
+// "grid" CTAs striding over the level's nodes, "npw" nodes a warp) on host threads, one
+// std::thread per CUDA thread, over inputs read from a case directory, and writes the caches and
+// the node arena back there.  Test infrastructure: it checks the kernels' barriers (every thread
+// reaches each one), their memory accesses (AddressSanitizer) and their results, without a GPU.
 //
 // usage: emu_extend <case dir>
 //   <dir>/params.txt  key value lines (scalars); "row_off", "slots", "span" lines (kMaxLevels+1
@@ -17,7 +18,7 @@
 #include "extend_extracted.h"
 
 namespace emu {
-thread_local int t_tid, t_block, t_crank, t_cs;
+thread_local int t_tid, t_block, t_crank, t_cs, t_grid = 1;
 thread_local long t_cluster_gen = -1;
 thread_local unsigned char *t_smem;
 std::vector<unsigned char *> g_cluster_smem;
@@ -62,10 +63,10 @@ void write_bin(const std::string &path, const std::vector<T> &v) {
   f.write(reinterpret_cast<const char *>(v.data()), (std::streamsize)(v.size() * sizeof(T)));
 }
 
-template <bool kPaged>
-void run_block(const ExtendArgs &a, int block) {
+template <typename Kernel>
+void run_block(Kernel kernel, size_t smem_bytes, int block, int grid) {
   using namespace emu;
-  std::vector<unsigned char> smem(kExtendSmem, 0xAB);
+  std::vector<unsigned char> smem(smem_bytes, 0xAB);
   g_smem_bytes = smem.size();
   g_cluster_smem.assign(1, smem.data());
   g_cta_bar = std::vector<TBarrier>(1);
@@ -81,8 +82,9 @@ void run_block(const ExtendArgs &a, int block) {
       t_crank = 0;
       t_cs = 1;
       t_block = block;
+      t_grid = grid;
       t_smem = smem.data();
-      extend_kernel<kPaged>(a);
+      kernel();
       g_where[t].line = -1;
       g_where[t].what = "exited";
     });
@@ -146,11 +148,55 @@ int main(int argc, char **argv) {
     a.span[l] = lists["span"].at(l);
   }
   const int blocks = (int)kv["batch"] * a.hkv;
-  for (int blk = 0; blk < blocks; ++blk) {
-    if (paged)
-      run_block<true>(a, blk);
-    else
-      run_block<false>(a, blk);
+  if ((int)kv["mode"] == 1) {  // the whole build, level by level, over `length` tokens
+    const int64_t length = (int64_t)kv["length"];
+    const int npw = (int)kv["npw"], grid_cap = (int)kv["grid"];
+    for (int l = 1; l <= a.levels; ++l) {
+      BuildArgs g = {};
+      const bool from_tokens = l == 1;
+      g.src_k = from_tokens ? ktok.data() : knode.data();
+      g.src_v = from_tokens ? vtok.data() : vnode.data();
+      g.src_row_off = from_tokens ? 0 : a.row_off[l - 1];
+      g.src_slots = a.slots[l - 1];
+      g.dst_k = knode.data();
+      g.dst_v = vnode.data();
+      g.dst_row_off = a.row_off[l];
+      g.dst_slots = a.slots[l];
+      g.span_prev = a.span[l - 1];
+      g.n_prev = (length + g.span_prev - 1) / g.span_prev;
+      g.length = length;
+      g.j0 = 0;
+      g.nj = (length + a.span[l] - 1) / a.span[l];
+      g.b = a.b;
+      g.bh = blocks;
+      g.hkv = a.hkv;
+      g.span = a.span[l];
+      g.seq_len = a.seq_len;
+      g.pages = from_tokens ? a.pages : nullptr;
+      g.page_shift = a.page_shift;
+      g.pages_per_seq = paged ? a.capacity >> a.page_shift : 0;
+      g.num_pages = a.num_pages;
+      g.pooler = pooler.data();
+      const int64_t per_block = (int64_t)kBuildWarps * npw;
+      const int grid = (int)std::min<int64_t>((g.bh * g.nj + per_block - 1) / per_block, grid_cap);
+      for (int blk = 0; blk < grid; ++blk) {
+        if (npw == 1 && g.pages)
+          run_block([&] { build_level_kernel<kFewNodes, true>(g); }, build_smem(kFewNodes), blk, grid);
+        else if (npw == 1)
+          run_block([&] { build_level_kernel<kFewNodes, false>(g); }, build_smem(kFewNodes), blk, grid);
+        else if (g.pages)
+          run_block([&] { build_level_kernel<kNodesPerWarp, true>(g); }, build_smem(kNodesPerWarp), blk, grid);
+        else
+          run_block([&] { build_level_kernel<kNodesPerWarp, false>(g); }, build_smem(kNodesPerWarp), blk, grid);
+      }
+    }
+  } else {
+    for (int blk = 0; blk < blocks; ++blk) {
+      if (paged)
+        run_block([&] { extend_kernel<true>(a); }, kExtendSmem, blk, blocks);
+      else
+        run_block([&] { extend_kernel<false>(a); }, kExtendSmem, blk, blocks);
+    }
   }
   write_bin(dir + "/k_tok_out.bin", ktok);
   write_bin(dir + "/v_tok_out.bin", vtok);

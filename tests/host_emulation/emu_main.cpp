@@ -17,7 +17,7 @@
 #include "lean_extracted.h"
 
 namespace emu {
-thread_local int t_tid, t_block, t_crank, t_cs;
+thread_local int t_tid, t_block, t_crank, t_cs, t_grid = 1;
 thread_local long t_cluster_gen = -1;
 thread_local unsigned char *t_smem;
 std::vector<unsigned char *> g_cluster_smem;

@@ -1,4 +1,4 @@
-"""The append kernel's own source, run on host threads against the oracle (no GPU).
+"""The append and level-build kernels' own source, run on host threads against the oracle (no GPU).
 
 tests/host_emulation cuts the append kernel (one CTA per (sequence, KV head) that copies the
 new tokens and rebuilds the nodes over them, level by level) out of the build source and
@@ -7,7 +7,9 @@ per CUDA thread, real rendezvous for every __syncthreads, and AddressSanitizer. 
 before the append is the oracle's, laid out in the library's arena; after it, the token
 slots must hold the new rows bit for bit and every node row must meet the node-row parity
 bar against the oracle's tree over the longer cache — for equal lengths, per-sequence
-lengths and a paged token cache.
+lengths and a paged token cache.  The level-build kernel runs the same way over every level
+(a grid that strides over the level's nodes, or a node per warp), its node rows held to the
+oracle's trees, with per-sequence lengths and a paged cache too.
 """
 
 import math
@@ -166,3 +168,76 @@ def test_append_with_per_sequence_lengths(emu_bin, tmp_path):
 @pytest.mark.parametrize("P", [1, 16])
 def test_append_into_a_paged_cache(emu_bin, tmp_path, P):
     _run(emu_bin, tmp_path, [600, 301], 1, 5, 4, P=P, per_seq=True, seed=P)
+
+
+def _run_build(emu_bin, tmp_path, lens, hkv, b, npw, grid, P=None, per_seq=False, seed=3):
+    """The level-build kernel over every level (grid-stride over `grid` CTAs, `npw` nodes a
+    warp) on the CPU; each sequence's node rows against the oracle's tree over its tokens."""
+    B, L = len(lens), max(lens)
+    cap = -(-L // P) * P if P else L
+    inp = I.random_case(B, L, hkv, hkv * 4, 0, seed=seed, capacity=cap)
+    kb, vb = bits(inp["k_tok"]), bits(inp["v_tok"])
+    pooler = inp["pooler"].double().numpy()
+    p = R.params(num_kv_heads=hkv, num_q_heads=hkv * 4, branching=b, top_k=2)
+    node_rows, levels_cap, offs = R.tree_layout(p, B, cap)
+    slots = [cap] + [math.ceil(cap / b ** lv) for lv in range(1, levels_cap + 1)]
+    prm = dict(mode=1, length=L, npw=npw, grid=grid, batch=B, hkv=hkv, b=b, capacity=cap, at=0, chunk=0,
+               levels=len(O.level_counts(L, b)) - 1, page_shift=0, num_pages=0)
+    k_in, v_in, pages = kb, vb, None
+    if P:
+        pps = cap // P
+        rng = np.random.default_rng(seed)
+        n_pages = B * pps + 3
+        pages = rng.permutation(n_pages)[:B * pps].astype(np.int32).reshape(B, pps)
+        prm.update(page_shift=int(math.log2(P)), num_pages=n_pages)
+        k_in = rng.integers(0, 1 << 16, size=(n_pages, hkv, P, 128), dtype=np.uint16)
+        v_in = k_in.copy()
+        for s in range(B):
+            for j in range(pps):
+                k_in[pages[s, j]] = kb[s, :, j * P:(j + 1) * P]
+                v_in[pages[s, j]] = vb[s, :, j * P:(j + 1) * P]
+    d = tmp_path / f"build_{B}_{hkv}_{L}_{b}_{npw}_{grid}_{P}_{int(per_seq)}"
+    d.mkdir()
+    span = [min(b ** lv, 1 << 62) for lv in range(R.MAX_LEVELS + 1)]
+    with open(d / "params.txt", "w") as f:
+        for key, val in prm.items():
+            f.write(f"{key} {val}\n")
+        f.write("row_off " + " ".join(str(offs[i] if i <= levels_cap else 0) for i in range(R.MAX_LEVELS + 1)) + "\n")
+        f.write("slots " + " ".join(str(slots[i] if i <= levels_cap else 0) for i in range(R.MAX_LEVELS + 1)) + "\n")
+        f.write("span " + " ".join(str(x) for x in span) + "\n")
+        if per_seq:
+            f.write("seq_len " + " ".join(str(n) for n in lens) + "\n")
+        if pages is not None:
+            f.write("pages " + " ".join(str(x) for x in pages.reshape(-1)) + "\n")
+    zeros = np.zeros((max(node_rows, 1), 128), np.uint16)
+    for name, arr in (("k_tok", k_in), ("v_tok", v_in), ("k_node", zeros), ("v_node", zeros),
+                      ("k_new", np.zeros(0, np.uint16)), ("v_new", np.zeros(0, np.uint16))):
+        np.ascontiguousarray(arr, dtype=np.uint16).tofile(d / f"{name}.bin")
+    np.ascontiguousarray(inp["pooler"].numpy(), dtype=np.float32).tofile(d / "pooler.bin")
+    r = subprocess.run([emu_bin, str(d)], capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, (r.stdout[-2000:], r.stderr[-4000:])
+    kn_out = np.fromfile(d / "k_node_out.bin", np.uint16).reshape(zeros.shape)
+    vn_out = np.fromfile(d / "v_node_out.bin", np.uint16).reshape(zeros.shape)
+    mism = total = 0
+    for s, n in enumerate(lens):
+        if n == 0:
+            continue
+        for h in range(hkv):
+            t = O.build_tree(O.bf16_bits_to_f64(kb[s, h, :n]), O.bf16_bits_to_f64(vb[s, h, :n]), pooler, b)
+            for lv in range(1, t.top + 1):
+                r0 = offs[lv] + (s * hkv + h) * slots[lv]
+                cnt = t.keys[lv].shape[0]
+                for got, want in ((kn_out[r0:r0 + cnt], t.keys[lv]), (vn_out[r0:r0 + cnt], t.values[lv])):
+                    a, c = check_node_rows(got, want)
+                    mism += a
+                    total += c
+    assert total > 0 and mism <= total * 1e-2
+
+
+@pytest.mark.parametrize("npw,grid", [(8, 2), (1, 1000)])  # a grid that strides, and a node per warp
+def test_level_build_matches_oracle(emu_bin, tmp_path, npw, grid):
+    _run_build(emu_bin, tmp_path, [1000, 1000], 2, 4, npw, grid)
+
+
+def test_level_build_with_per_sequence_lengths_and_pages(emu_bin, tmp_path):
+    _run_build(emu_bin, tmp_path, [700, 0, 301, 64], 1, 4, 8, 3, P=8, per_seq=True)
