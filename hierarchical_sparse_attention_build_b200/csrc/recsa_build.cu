@@ -348,7 +348,7 @@ __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendA
   for (int i = 0; i < kPieces; ++i) w[i] = __ldg(reinterpret_cast<const float4 *>(a.pooler) + tid + i * kExtendThreads);
   {
     const int64_t s = bhi / a.hkv;
-    for (int e = tid; e < a.chunk * 16; e += kExtendThreads) {  // 16 pieces a row
+    for (int64_t e = tid; e < (int64_t)a.chunk * 16; e += kExtendThreads) {  // 16 pieces a row
       const int64_t src = ((s * a.chunk + (e >> 4)) * a.hkv + h) * 16 + (e & 15);
       const int64_t row = tok_row(at + (e >> 4));
       if (row < 0) continue;

@@ -44,7 +44,9 @@ def shard_params(p, rank: int, world: int):
 
 
 def shard_cache(x: torch.Tensor, h0: int, h1: int) -> torch.Tensor:
-    """A token cache [B][Hkv][capacity][128] -> this block's own contiguous cache."""
+    """A token cache [B][Hkv][capacity][128] -> this block's own contiguous cache.  A paged
+    pool [num_pages][Hkv][page_size][128] shards the same way (heads are its second axis), and
+    every rank keeps the whole page table."""
     return x[:, h0:h1].contiguous()
 
 
