@@ -296,7 +296,9 @@ constexpr int kExtendThreads = 2 * kD;  // one thread per key dimension and per 
 constexpr int kHalfK = kD / 2;          // W columns held by each thread of a dimension
 // W^T staged as Wt[k][o ^ (k / 4 % 32)]: the coalesced row loads (a warp reads one W row)
 // and the per-thread row reads both hit 32 distinct banks.
-constexpr size_t kExtendSmem = (size_t)(kD * kD + 2 * kD) * sizeof(float);
+// W^T staging, the key mean, the first half of the key, and per level the rebuilt node range
+// [j0, j1) and the node count of the level below
+constexpr size_t kExtendSmem = (size_t)(kD * kD + 2 * kD) * sizeof(float) + 3 * (kMaxLevels + 1) * sizeof(int64_t);
 
 // x / y and ceil(x / y) for x >= 0, y >= 1, in 32 bits whenever the operands fit (a 64-bit
 // division is a long instruction sequence; lengths and spans of real trees fit 32 bits).
@@ -317,6 +319,9 @@ __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendA
   float *Wt = smem_f;               // swizzled W^T (staging only)
   float *mean = smem_f + kD * kD;   // the node's key mean
   float *part = mean + kD;          // key outputs after k < 64
+  int64_t *lv_j0 = reinterpret_cast<int64_t *>(part + kD);  // per level: nodes [j0, j1) rebuilt,
+  int64_t *lv_j1 = lv_j0 + (kMaxLevels + 1);                 // the level below's node count
+  int64_t *lv_np = lv_j1 + (kMaxLevels + 1);
   const int tid = threadIdx.x;
   const int64_t bhi = blockIdx.x;   // (sequence, head)
   const int d = tid & (kD - 1);
@@ -328,11 +333,14 @@ __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendA
   while (t_new < a.levels && a.span[t_new + 1] < length) ++t_new;
   while (t_old < t_new && a.span[t_old + 1] < at) ++t_old;
   // level l rebuilds nodes [j0, j1): those whose spans meet the new tokens (a level that
-  // becomes new is built whole)
-  auto node_range = [&](int l, int64_t *j0, int64_t *j1) {
-    *j0 = l <= t_old ? div_nn(at, a.span[l]) : 0;
-    *j1 = ceil_div_nn(length, a.span[l]);
-  };
+  // becomes new is built whole); the first warp works the levels out side by side, once,
+  // rather than every thread on the walk's dependent path
+  if (tid < 32)
+    for (int l = tid + 1; l <= t_new; l += 32) {
+      lv_j0[l] = l <= t_old ? div_nn(at, a.span[l]) : 0;
+      lv_j1[l] = ceil_div_nn(length, a.span[l]);
+      lv_np[l] = ceil_div_nn(length, a.span[l - 1]);
+    }
   // token t of this (sequence, head): row tok_base + tok_row(t), -1 for a page outside the pool
   const int64_t h = bhi % a.hkv;
   const int64_t tok_base = kPaged ? (h << a.page_shift) * kD : bhi * a.capacity * kD;
@@ -357,27 +365,22 @@ __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendA
       reinterpret_cast<uint4 *>(a.v_tok)[dst] = __ldg(a.v_new + src);
     }
   }
+  __syncthreads();  // the level ranges are in place, and the appended rows are read below by other threads
   // every child row the walk reads above level 1, into L2 ahead of the dependent levels
   // (K and V, two 128-byte lines each)
   for (int l = 2; l <= t_new; ++l) {
-    const int64_t n_prev = ceil_div_nn(length, a.span[l - 1]);
-    int64_t j0, j1;
-    node_range(l, &j0, &j1);
-    const int64_t c0 = j0 * a.b, c1 = min(j1 * a.b, n_prev);
+    const int64_t c0 = lv_j0[l] * a.b, c1 = min(lv_j1[l] * a.b, lv_np[l]);
     const int64_t base = (a.row_off[l - 1] + bhi * a.slots[l - 1]) * kD;
     for (int64_t e = tid; e < (c1 - c0) * 4; e += kExtendThreads)
       prefetch_l2(((e & 2) ? a.v_node : a.k_node) + base + (c0 + (e >> 2)) * kD + (e & 1) * (kD / 2));
   }
-  __syncthreads();  // the appended rows are read below by other threads
 
   float wr[kHalfK];  // W[d][64 * is_v + i]
   bool w_ready = false;
   const int kbase = is_v ? kHalfK : 0;
   for (int l = 1; l <= t_new; ++l) {
     const int64_t span_prev = a.span[l - 1];
-    const int64_t n_prev = ceil_div_nn(length, span_prev);
-    int64_t j0, j1;
-    node_range(l, &j0, &j1);
+    const int64_t n_prev = lv_np[l], j0 = lv_j0[l], j1 = lv_j1[l];
     const uint16_t *src = l == 1 ? (is_v ? a.v_tok : a.k_tok) + tok_base
                                  : (is_v ? a.v_node : a.k_node) + (a.row_off[l - 1] + bhi * a.slots[l - 1]) * kD;
     uint16_t *dk = a.k_node + (a.row_off[l] + bhi * a.slots[l]) * kD;
