@@ -180,3 +180,28 @@ def test_paged_other_group_sizes_equal_contiguous(G, b, P, kernel, cluster_size)
     x.assert_same_trees()
     a, c = x.decode_both(x.inp["q"], kernel, cluster_size)
     assert torch.equal(a, c)
+
+
+@pytest.mark.parametrize("pinned", [True, False])
+def test_host_buffer_and_no_alloc_decode_over_paged_varlen_cache(pinned):
+    """recsa_decode_host and recsa_decode_no_alloc over a paged cache with per-sequence lengths
+    give recsa_decode's bits."""
+    x = Pair(3, 2, 4, 800, 4, 2, 16, seed=31, queries=2, lens=[800, 5, 333])
+    x.build()
+    q = x.inp["q"].cuda().contiguous()
+    want = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    R.decode(x.p, x.g, q, want, x.ws)
+    R.check_device_errors(x.ws)
+    q_host = x.inp["q"].contiguous()
+    out_host = torch.empty(q.shape, dtype=torch.float32)
+    if pinned:
+        q_host, out_host = q_host.pin_memory(), out_host.pin_memory()
+    q_dev, out_dev = torch.empty_like(q), torch.empty_like(want)
+    R.decode_host(x.p, x.g, q_host, out_host, q_dev, out_dev, x.ws)
+    torch.cuda.synchronize()
+    R.check_device_errors(x.ws)
+    assert torch.equal(out_host, want.cpu())
+    got = torch.empty_like(want)
+    R.decode_no_alloc(x.p, x.g, q, got)
+    torch.cuda.synchronize()
+    assert torch.equal(got, want)
