@@ -100,6 +100,7 @@ def _load() -> ctypes.CDLL:
         "recsa_decode": [P, T, vp, i32, vp, i32, vp, sz, D, vp],
         "recsa_decode_host": [P, T, vp, i32, vp, i32, vp, vp, vp, sz, D, vp],
         "recsa_append": [P, T, vp, vp, i32, vp],
+        "recsa_decode_step": [P, T, vp, vp, vp, vp, i32, vp, sz, vp],
         "recsa_prefill_chunk": [P, T, vp, vp, vp, i32, vp, i32, vp, sz, D, vp],
         "recsa_check_device_errors": [vp, vp],
         "recsa_decode_no_alloc": [P, T, vp, i32, vp, i32, vp],
@@ -268,6 +269,17 @@ def append(p: Params, tree: RecsaTree, k_new: torch.Tensor, v_new: torch.Tensor,
         assert t.dtype == torch.bfloat16 and t.is_contiguous()
     _check(_lib.recsa_append(ctypes.byref(p), ctypes.byref(tree.c), _ptr(k_new), _ptr(v_new), k_new.shape[1],
                              _stream(stream)))
+
+
+def decode_step(p: Params, tree: RecsaTree, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor,
+                out: torch.Tensor, ws: Workspace, stream=None) -> None:
+    """recsa_decode_step: append one token per sequence at its device length, advance the
+    lengths, decode the token's query; graph-capturable (needs tree.seq_len)."""
+    for t in (k_new, v_new, q):
+        assert t.dtype == torch.bfloat16 and t.is_contiguous() and t.shape[1] == 1
+    _check(_lib.recsa_decode_step(ctypes.byref(p), ctypes.byref(tree.c), _ptr(k_new), _ptr(v_new), _ptr(q),
+                                  _ptr(out), int(out.dtype == torch.float32), _ptr(ws.buf), ws.nbytes,
+                                  _stream(stream)))
 
 
 def prefill_chunk(p: Params, tree: RecsaTree, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor,

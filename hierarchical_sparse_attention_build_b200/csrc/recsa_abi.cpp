@@ -393,11 +393,57 @@ RECSA_API recsa_status recsa_append(const recsa_params *params, recsa_tree *tree
   s = extend_tree(g, *tree, k_new, v_new, L, count, stream);
   if (s != RECSA_OK) return s;
   if (tree->seq_len) {
-    const int rc = launch_advance_lengths(tree->seq_len, tree->batch, count, stream);
+    const int rc = launch_advance_lengths(tree->seq_len, tree->batch, count, L + count, stream);
     if (rc != 0) return cuda_fail(rc, "advance of the sequence lengths");
   }
   tree->length = L + count;
   return RECSA_OK;
+}
+
+RECSA_API recsa_status recsa_decode_step(const recsa_params *params, const recsa_tree *tree, const void *k_new,
+                                         const void *v_new, const void *q, void *out, int32_t out_is_fp32, void *ws,
+                                         size_t ws_bytes, recsa_stream_t stream) {
+  recsa_status s = check_params(params);
+  if (s != RECSA_OK) return s;
+  TreeGeom g;
+  s = check_tree(params, tree, &g);
+  if (s != RECSA_OK) return s;
+  if (!tree->seq_len) return fail(RECSA_ERR_INVALID_ARGUMENT, "a decode step needs per-sequence lengths (tree->seq_len)");
+  if (!k_new || !v_new || !q || !out) return fail(RECSA_ERR_INVALID_ARGUMENT, "k_new, v_new, q or out is NULL");
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(q) || !aligned16(out))
+    return fail(RECSA_ERR_INVALID_ARGUMENT, "k_new, v_new, q or out is not 16-byte aligned");
+  s = check_ws(params, tree, ws, ws_bytes);
+  if (s != RECSA_OK) return s;
+  // every bound comes from the capacity, none from the current lengths
+  const int64_t cap = tree->capacity;
+  const int64_t mc = max_candidates(params, cap, false);
+  if (mc > kMaxCand)
+    return fail(RECSA_ERR_UNSUPPORTED, "up to %lld candidates per level > %d", (long long)mc, kMaxCand);
+  uint32_t *err = &reinterpret_cast<WsHeader *>(ws)->err;
+  int rc = launch_extend(g, *tree, k_new, v_new, cap - 1, 1, levels_for(cap, g.b), stream, err);
+  if (rc != 0) return cuda_fail(rc, "append and path update");
+  rc = launch_advance_lengths(tree->seq_len, tree->batch, 1, cap, stream);
+  if (rc != 0) return cuda_fail(rc, "advance of the sequence lengths");
+  AttendLaunch l;
+  l.geom = g;
+  l.tree = *tree;
+  l.q = q;
+  l.out = out;
+  l.out_fp32 = out_is_fp32 ? 1 : 0;
+  l.num_queries = 1;
+  l.length = cap;
+  l.causal = 0;
+  l.group = params->num_q_heads / params->num_kv_heads;
+  l.top_k = params->top_k;
+  l.scale = params->softmax_scale > 0.f ? params->softmax_scale : 1.0f / std::sqrt((float)kD);
+  l.ws = ws;
+  l.table_rows_needed = (int)mc + 1;
+  l.max_cand = (int)((mc + 31) / 32 * 32);
+  l.cluster_size = 0;
+  l.kernel = 0;
+  l.debug = nullptr;
+  rc = launch_attend(l, stream);
+  return rc != 0 ? cuda_fail(rc, "decode attend") : RECSA_OK;
 }
 
 RECSA_API recsa_status recsa_prefill_chunk(const recsa_params *params, recsa_tree *tree, const void *k_new,
@@ -451,7 +497,7 @@ RECSA_API recsa_status recsa_prefill_chunk(const recsa_params *params, recsa_tre
   int rc = launch_attend(l, stream);
   if (rc != 0) return cuda_fail(rc, "prefill attend");
   if (tree->seq_len) {
-    rc = launch_advance_lengths(tree->seq_len, tree->batch, chunk, stream);
+    rc = launch_advance_lengths(tree->seq_len, tree->batch, chunk, L2, stream);
     if (rc != 0) return cuda_fail(rc, "advance of the sequence lengths");
   }
   tree->length = L2;

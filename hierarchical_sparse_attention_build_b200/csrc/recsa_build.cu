@@ -285,6 +285,7 @@ struct ExtendArgs {
   const int64_t *seq_len;       // per-sequence lengths before the append (NULL: all `at`)
   const int32_t *pages;         // paged token cache: the page table (NULL: contiguous)
   int32_t page_shift, num_pages;
+  uint32_t *err;                // optional error word: a sequence without room is flagged
   int64_t capacity;
   int64_t at;                   // first new slot (the length before the append; the longest one)
   int32_t chunk, hkv, b, levels;  // levels = T(at + chunk)
@@ -327,7 +328,14 @@ __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendA
   const int d = tid & (kD - 1);
   const bool is_v = tid >= kD;
   // this sequence's length before (at) and after (length) the append, and its levels
-  const int64_t at = a.seq_len ? min(max(a.seq_len[bhi / a.hkv], (int64_t)0), a.at) : a.at;
+  int64_t at = a.at;
+  if (a.seq_len) {  // a sequence outside [0, at] (no room for the chunk) is left as it is
+    at = a.seq_len[bhi / a.hkv];
+    if (at < 0 || at > a.at) {
+      if (a.err && tid == 0) atomicOr(a.err, kErrIndex);
+      return;  // the whole CTA: every thread reads the same length
+    }
+  }
   const int64_t length = at + a.chunk;
   int t_old = 0, t_new = 0;  // T(n) = #{l >= 1 : b^l < n}
   while (t_new < a.levels && a.span[t_new + 1] < length) ++t_new;
@@ -604,8 +612,9 @@ int launch_build_level(const TreeGeom &g, const recsa_tree &t, int level, int64_
 }
 
 int launch_extend(const TreeGeom &g, const recsa_tree &t, const void *k_new, const void *v_new, int64_t at,
-                  int chunk, int levels, void *stream) {
+                  int chunk, int levels, void *stream, uint32_t *err) {
   ExtendArgs a;
+  a.err = err;
   a.k_new = reinterpret_cast<const uint4 *>(k_new);
   a.v_new = reinterpret_cast<const uint4 *>(v_new);
   a.k_tok = reinterpret_cast<uint16_t *>(t.k_tok);
@@ -636,14 +645,16 @@ int launch_extend(const TreeGeom &g, const recsa_tree &t, const void *k_new, con
   return (int)cudaGetLastError();
 }
 
-__global__ void advance_lengths_kernel(int64_t *seq_len, int batch, int64_t count) {
+// seq_len[s] += count, held to `limit` (a sequence the append skipped stays where it was).
+__global__ void advance_lengths_kernel(int64_t *seq_len, int batch, int64_t count, int64_t limit) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < batch) seq_len[i] += count;
+  if (i < batch && seq_len[i] >= 0 && seq_len[i] + count <= limit) seq_len[i] += count;
 }
 
-int launch_advance_lengths(int64_t *seq_len, int batch, int64_t count, void *stream) {
+int launch_advance_lengths(int64_t *seq_len, int batch, int64_t count, int64_t limit, void *stream) {
   const int threads = 128;
-  advance_lengths_kernel<<<(batch + threads - 1) / threads, threads, 0, (cudaStream_t)stream>>>(seq_len, batch, count);
+  advance_lengths_kernel<<<(batch + threads - 1) / threads, threads, 0, (cudaStream_t)stream>>>(seq_len, batch, count,
+                                                                                               limit);
   return (int)cudaGetLastError();
 }
 

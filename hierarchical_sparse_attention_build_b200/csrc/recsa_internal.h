@@ -59,9 +59,10 @@ int launch_append(const TreeGeom &g, const recsa_tree &t, const void *k_new, con
 // and rebuild the nodes over them, all levels in one launch (a CTA per (sequence, head)
 // walks up the levels).  levels = T of the longest new length.
 int launch_extend(const TreeGeom &g, const recsa_tree &t, const void *k_new, const void *v_new, int64_t at,
-                  int chunk, int levels, void *stream);
-// seq_len[s] += count for every sequence (queued after the kernels that read the old lengths).
-int launch_advance_lengths(int64_t *seq_len, int batch, int64_t count, void *stream);
+                  int chunk, int levels, void *stream, uint32_t *err = nullptr);
+// seq_len[s] += count for every sequence whose new length stays within `limit` (queued after
+// the kernels that read the old lengths).
+int launch_advance_lengths(int64_t *seq_len, int batch, int64_t count, int64_t limit, void *stream);
 
 struct AttendLaunch {
   TreeGeom geom;

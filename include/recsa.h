@@ -231,6 +231,22 @@ RECSA_API recsa_status recsa_decode_host(const recsa_params *params, const recsa
 RECSA_API recsa_status recsa_append(const recsa_params *params, recsa_tree *tree, const void *k_new,
                                     const void *v_new, int32_t count, recsa_stream_t stream);
 
+/* One decode step of a serving loop whose lengths live on the device: for every sequence s,
+ * append one token (k_new, v_new: bf16 [batch][1][Hkv][128]) at slot seq_len[s] and update
+ * the tree over it (as recsa_append), advance seq_len[s] by one, and decode that token's
+ * query (q: bf16 [batch][1][Hq][128]; out as in recsa_decode) over its seq_len[s] tokens.
+ * Not in the abstract: the plumbing of a decode loop.  Every kernel parameter comes from
+ * the tree's capacity and its arrays, none from the current lengths, so the call can be
+ * captured once into a CUDA graph and the graph replayed step after step (the caller writes
+ * each step's k_new, v_new and q into the same buffers before a replay).  Needs
+ * tree->seq_len (else RECSA_ERR_INVALID_ARGUMENT); tree->length is neither read nor
+ * written.  A sequence with no room left (seq_len[s] == capacity) is not appended to, keeps
+ * its length, and is flagged in the workspace error word (RECSA_ERR_DEVICE_CHECK); its query
+ * is decoded over its tokens as they are. */
+RECSA_API recsa_status recsa_decode_step(const recsa_params *params, const recsa_tree *tree, const void *k_new,
+                                         const void *v_new, const void *q, void *out, int32_t out_is_fp32,
+                                         void *ws, size_t ws_bytes, recsa_stream_t stream);
+
 /* Causal prefill of a chunk of `chunk` tokens at positions L .. L+chunk-1
  * (L = tree->length): appends k_new / v_new to the token caches, rebuilds the tree
  * nodes those tokens touch (and any level that becomes new), then attends query i

@@ -29,7 +29,8 @@ def test_library_exports_every_declared_symbol():
     names = declared_functions()
     assert set(names) == {"recsa_tree_layout", "recsa_workspace_size", "recsa_workspace_init", "recsa_build_tree",
                           "recsa_decode", "recsa_prefill_chunk", "recsa_check_device_errors", "recsa_status_string",
-                          "recsa_last_error", "recsa_decode_no_alloc", "recsa_decode_host", "recsa_append"}, names
+                          "recsa_last_error", "recsa_decode_no_alloc", "recsa_decode_host", "recsa_append",
+                          "recsa_decode_step"}, names
     for n in names:
         assert hasattr(lib, n), n
         assert ctypes.cast(getattr(lib, n), ctypes.c_void_p).value
@@ -193,6 +194,19 @@ def test_paged_cache_arguments_rejected(kw):
     d = dict(length=100, page_table=FAKE, page_size=8, num_pages=16)
     d.update(kw)
     assert lib.recsa_build_tree(ctypes.byref(p), ctypes.byref(_tree(**d)), None) == INVALID
+
+
+def test_decode_step_checks_everything_before_queuing():
+    p = _p()
+    ws = R.workspace_size(p, 4096)
+    call = lambda t, **kw: lib.recsa_decode_step(ctypes.byref(p), ctypes.byref(t), kw.get("k", FAKE), kw.get("v", FAKE),
+                                                 kw.get("q", FAKE), kw.get("out", FAKE), 1, FAKE, kw.get("ws", ws), None)
+    assert call(_tree(length=100)) == INVALID                     # no per-sequence lengths
+    with_len = _tree(length=100, seq_len=FAKE)
+    assert call(with_len, q=0) == INVALID
+    assert call(with_len, k=FAKE + 4) == INVALID
+    assert call(with_len, ws=10) == WS_SMALL
+    assert call(_tree(length=100, seq_len=FAKE + 4)) == INVALID   # misaligned lengths
 
 
 def test_layout_and_build_reject_bad_input():
