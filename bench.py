@@ -305,13 +305,13 @@ def leg_decode_loop(R, timer, args, dist_on):
     w = I.WORKLOADS["decode_1m"]
     warmup, steps = 4, 64 if not args.quick else 16
     per_leg = warmup + steps
-    inp = I.decode_inputs(w, device="cuda", capacity=w.length + 2 * per_leg + 8)
+    inp = I.decode_inputs(w, device="cuda", capacity=w.length + 3 * per_leg + 8)
     p = R.params(num_kv_heads=w.kv_heads, num_q_heads=w.q_heads, branching=w.branching, top_k=w.top_k)
     tree, ws = make_tree(R, p, inp, w.length)
     g = torch.Generator(device="cuda").manual_seed(91)
     B, Hkv, Hq = w.batch, w.kv_heads, w.q_heads
     toks = [tuple(torch.randn(B, 1, h, 128, generator=g, device="cuda").to(torch.bfloat16) for h in (Hkv, Hkv, Hq))
-            for _ in range(2 * per_leg)]
+            for _ in range(3 * per_leg + 2)]
     out = torch.empty(B, 1, Hq, 128, dtype=torch.bfloat16, device="cuda")
     nxt = [0]
 
@@ -331,13 +331,57 @@ def leg_decode_loop(R, timer, args, dist_on):
     per, _ = timer.run(chunk_of_one, steps, warmup)
     t_chunk = max_over_ranks(sum(per), dist_on) / steps
     R.check_device_errors(ws)
-    del tree, ws, inp
+
+    # the same step as recsa_decode_step replayed from one CUDA graph: lengths on the device,
+    # each step's token and query written into fixed buffers before the replay (untimed, as
+    # the model would write them)
+    seq_len = torch.full((B,), tree.length, dtype=torch.int64, device="cuda")
+    gtree = R.RecsaTree(p, inp["k_tok"], inp["v_tok"], inp["pooler"], tree.length, k_node=tree.k_node,
+                        v_node=tree.v_node, seq_len=seq_len)
+    kbuf, vbuf, qbuf = (torch.empty(B, 1, h, 128, dtype=torch.bfloat16, device="cuda") for h in (Hkv, Hkv, Hq))
+
+    def fill():
+        kn, vn, qn = toks[nxt[0]]
+        nxt[0] += 1
+        kbuf.copy_(kn)
+        vbuf.copy_(vn)
+        qbuf.copy_(qn)
+
+    fill()
+    R.decode_step(p, gtree, kbuf, vbuf, qbuf, out, ws)  # first launches outside the capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(graph, stream=side):
+        R.decode_step(p, gtree, kbuf, vbuf, qbuf, out, ws)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(warmup + steps):
+        fill()
+        timer.flush()
+        if i >= warmup:
+            ev[i - warmup][0].record(stream)
+        graph.replay()
+        if i >= warmup:
+            ev[i - warmup][1].record(stream)
+    torch.cuda.synchronize()
+    t_graph = max_over_ranks(sum(a.elapsed_time(b) / 1e3 for a, b in ev), dist_on) / steps
+    R.check_device_errors(ws)
+    del graph
+    del tree, gtree, ws, inp
     torch.cuda.empty_cache()
     return {"workload": f"decode_loop_1m: B={B}, L={w.length} + 1 token per sequence per step, Hq={Hq}, "
                         f"Hkv={Hkv}, b={w.branching}, k={w.top_k}",
             "tokens_per_s": B / t, "us_per_step": t * 1e6, "launches_per_step": 2,
             "note": "recsa_append (token slot + ancestor path of every (sequence, KV head), one launch) + "
                     "recsa_decode of the new token's query; L2 flushed before each step",
+            "graph_replay": {"us_per_step": t_graph * 1e6, "tokens_per_s": B / t_graph, "launches_per_step": 3,
+                             "note": "recsa_decode_step (append, length advance, decode) captured once into a CUDA "
+                                     "graph and replayed per step; L2 flushed before each replay (the eager calls "
+                                     "above are queued while that flush runs, so their launch cost is hidden here "
+                                     "too; the graph pays off when steps run back to back)"},
             "causal_chunk_of_1": {"us_per_step": t_chunk * 1e6, "launches_per_step": 2,
                                   "note": "recsa_prefill_chunk with C = 1: the same update, then the causal "
                                           "attend (the partial node on the query's path always expanded)"}}
