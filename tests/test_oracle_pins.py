@@ -141,6 +141,31 @@ def test_build_values_are_subtree_means_exact_mode():
                 assert tree.counts[lvl][j] == O.subtree_tokens(lvl, j, b, L)
 
 
+def test_appending_tokens_leaves_complete_nodes_unchanged():
+    # A node depends only on its subtree's tokens (its value is their mean; its key is W applied
+    # to its children's stored keys), so growing the cache from L to L + C changes no node whose
+    # span ends at or before L, and every node that does change meets [L, L + C) or lies on a
+    # level that did not exist.  The incremental update rebuilds exactly those nodes.
+    rng = np.random.default_rng(12)
+    w = np.linalg.qr(rng.standard_normal((128, 128)))[0]
+    for L, C, b in [(1000, 1, 4), (1023, 1, 4), (700, 40, 16), (255, 3, 2)]:
+        kt, vt = rng.standard_normal((L + C, 128)), rng.standard_normal((L + C, 128))
+        before = O.build_tree(kt[:L], vt[:L], w, b)
+        after = O.build_tree(kt, vt, w, b)
+        for lvl in range(1, after.top + 1):
+            span = b ** lvl
+            n_after = after.keys[lvl].shape[0]
+            n_before = before.keys[lvl].shape[0] if lvl <= before.top else 0
+            for j in range(n_after):
+                complete = (j + 1) * span <= L and j < n_before
+                same = (j < n_before and np.array_equal(before.keys[lvl][j], after.keys[lvl][j])
+                        and np.array_equal(before.values[lvl][j], after.values[lvl][j]))
+                if complete:
+                    assert same, (L, C, b, lvl, j)
+                else:  # the node holds a new token (or its level is new): it is rebuilt
+                    assert j * span < L + C and ((j + 1) * span > L or j >= n_before)
+
+
 def test_build_keys_closed_form_full_nodes():
     # Full nodes: K_l[j] = W^l (subtree token mean); with W = I it is the subtree mean.
     rng = np.random.default_rng(4)
