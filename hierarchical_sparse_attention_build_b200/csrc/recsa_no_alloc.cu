@@ -27,10 +27,41 @@ static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBy
 
 constexpr int kMaxDevices = 128;
 void *g_scratch_ptr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};
 std::mutex g_scratch_mu;
 
-// Device address of g_static_scratch on the current device, looked up on the first
-// call made with that device current.
+// Unique id of the calling thread's current CUDA context (0 when there is none, or when
+// the driver cannot say).  A device reset destroys the context, and the array with it;
+// the next context gets a new id, so an address kept from the old one is never reused.
+unsigned long long current_context_id() {
+  using GetCurrent = int (*)(void **);
+  using GetId = int (*)(void *, unsigned long long *);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(f);
+  });
+  void *ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != 0 || ctx == nullptr ||
+      get_id(ctx, &id) != 0)
+    return 0;
+  return id;
+}
+
+// Device address of g_static_scratch for the current device, looked up with
+// cudaGetSymbolAddress on the first call made with that device current and again only
+// when the device's context has changed since (a reset).  Without a context id the
+// address is looked up on every call.
 recsa_status static_scratch(void **out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -43,14 +74,17 @@ recsa_status static_scratch(void **out) {
     return RECSA_ERR_UNSUPPORTED;
   }
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (g_scratch_ptr[dev] == nullptr || ctx == 0 || g_scratch_ctx[dev] != ctx) {
     void *p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    e = cudaGetSymbolAddress(&p, g_static_scratch);  // also creates the context on a first call
     if (e != cudaSuccess || p == nullptr) {
+      g_scratch_ptr[dev] = nullptr;
       set_error("RECSA_ERR_CUDA: cudaGetSymbolAddress of the static scratch: %s", cudaGetErrorString(e));
       return RECSA_ERR_CUDA;
     }
     g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = current_context_id();
   }
   *out = g_scratch_ptr[dev];
   return RECSA_OK;

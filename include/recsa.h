@@ -270,7 +270,8 @@ RECSA_API recsa_status recsa_prefill_chunk(const recsa_params *params, recsa_tre
  * 256 KiB device array of the library, which every GPU that loads the library holds
  * until the process exits.
  *   - The first call made with a device current looks the array's address up on that
- *     device; make that first call before any stream capture.
+ *     device (and again after the device's context was re-created, e.g. by a reset);
+ *     make that first call before any stream capture.
  *   - Every call rewrites the array (table for its own parameters, error word cleared),
  *     so calls whose GPU work overlaps (other streams, other threads) race: order them
  *     on one stream.

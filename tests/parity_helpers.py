@@ -13,6 +13,8 @@ Comparison rules (the method's acceptance bar):
 
 from __future__ import annotations
 
+import os
+
 import numpy as np
 import torch
 
@@ -124,8 +126,15 @@ def gpu_selection(sel: np.ndarray, tile: int, top: int) -> list[list[int]]:
     return out
 
 
+# Every Stats made while a test runs is recorded under that test's id, so the end of the
+# session can report tiles, near-tie swaps and errors per configuration.
+REPORT: list[tuple[str, "Stats"]] = []
+
+
 class Stats:
-    def __init__(self):
+    def __init__(self, label: str | None = None):
+        test = os.environ.get("PYTEST_CURRENT_TEST", "").split(" (")[0]
+        REPORT.append((label or test or "untitled", self))
         self.tiles = 0
         self.near_ties = 0
         self.max_abs = 0.0

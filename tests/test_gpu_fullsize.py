@@ -3,7 +3,8 @@
 Every call runs in the launch shape the benchmark times (automatic kernel choice) over
 the whole batch; the oracle then rebuilds only the sampled (sequence, KV head) trees and
 checks their node rows, the sampled tiles' selections (exact up to validated near-ties)
-and outputs, and the tiles' row counts.
+and outputs, and the tiles' row counts.  The decode cases check every tile of one whole
+sequence (all of its KV heads) and a few heads of other sequences.
 """
 
 import numpy as np
@@ -75,16 +76,17 @@ def _decode_case(name, samples):
     return stats
 
 
+# every KV head (every tile) of one sequence, plus heads of other sequences
 def test_decode_131k_batch8():
-    _decode_case("decode_131k", [(0, 0), (3, 5), (7, 7)])
+    _decode_case("decode_131k", [(3, h) for h in range(8)] + [(0, 0), (7, 7)])
 
 
 def test_decode_1m_batch4_needles():
-    _decode_case("decode_1m", [(0, 0), (1, 3), (3, 7)])
+    _decode_case("decode_1m", [(1, h) for h in range(8)] + [(0, 0), (3, 7)])
 
 
 def test_build_and_decode_2m():
-    _decode_case("build_decode_2m", [(0, 2), (0, 6)])
+    _decode_case("build_decode_2m", [(0, h) for h in range(8)])
 
 
 def test_prefill_524k_chunk_8192():

@@ -428,3 +428,116 @@ def test_worked_example_causal_forced_partial_node():
     num = math.exp(s1) * vt[4:8].mean(0) + vt[0:4].sum(0) + vt[8] + vt[9]
     want = num / (math.exp(s1) + 6)
     assert np.abs(got[0] - want).max() < 1e-13
+
+
+def test_dense_attention_two_token_closed_form():
+    # keys A e_0 at position 0 and 0 at position 1, query e_0 at position 2: the pair
+    # (0, 64) turns 1 rad per position, so the first logit is scale * A * cos(2 - 0).
+    A = 5.0
+    keys = np.stack([_e(0, A), np.zeros(128)])
+    vals = np.stack([_e(1), _e(2)])
+    s0 = SCALE * A * math.cos(2.0)
+    want = (math.exp(s0) * _e(1) + _e(2)) / (math.exp(s0) + 1.0)
+    got = O.dense_attention(_e(0)[None, :], keys, vals, 2)
+    assert np.abs(got[0] - want).max() < 1e-14
+
+
+# --------------------------------------------------------------------------- whole-call drivers
+# The drivers slice the call's tensors into tiles: query heads g*G .. g*G+G-1 belong to
+# KV group g (the repeat-kv convention), decode queries sit at p = L, prefill query i
+# at p = L + i, and a chunk arrives as [B][C][Hkv][128].  Each is pinned here against
+# inputs whose right answer does not depend on the driver's own slicing.
+
+def _bf16_bits_of(x):
+    return O.f64_to_bf16_bits(np.asarray(x, dtype=np.float64))
+
+
+def test_decode_all_groups_query_heads_in_contiguous_blocks():
+    # every value row of (sequence s, KV head h) is the constant 10 s + h, so any softmax
+    # over that tree outputs exactly 10 s + h: output head j of sequence s must read
+    # 10 s + j // G.  An interleaved mapping (j % Hkv) or a swapped sequence fails.
+    B, Hkv, G, Q, L, b, k = 2, 2, 4, 3, 40, 4, 2
+    rng = np.random.default_rng(21)
+    kb = _bf16_bits_of(rng.standard_normal((B, Hkv, L, 128)))
+    vals = np.zeros((B, Hkv, L, 128))
+    for s in range(B):
+        for h in range(Hkv):
+            vals[s, h] = 10 * s + h
+    vb = _bf16_bits_of(vals)
+    qb = _bf16_bits_of(rng.standard_normal((B, Q, Hkv * G, 128)))
+    trees = O.build_all(kb, vb, np.eye(128), b, L)
+    out = O.decode_all(trees, qb, k)
+    for s in range(B):
+        for qi in range(Q):
+            for j in range(Hkv * G):
+                assert np.abs(out[s, qi, j] - (10 * s + j // G)).max() < 1e-12, (s, qi, j)
+
+
+def test_decode_all_topk_all_is_dense_per_query_head():
+    # k = all: each output head is dense RoPE attention of its own query row over its
+    # group's tokens at their positions, query at L (checked head by head).
+    B, Hkv, G, Q, L, b = 2, 3, 2, 2, 50, 4
+    rng = np.random.default_rng(22)
+    kb = _bf16_bits_of(rng.standard_normal((B, Hkv, L, 128)))
+    vb = _bf16_bits_of(rng.standard_normal((B, Hkv, L, 128)))
+    qb = _bf16_bits_of(rng.standard_normal((B, Q, Hkv * G, 128)) * 2)
+    out = O.decode_all(O.build_all(kb, vb, np.eye(128), b, L), qb, O.TOPK_ALL)
+    for s in range(B):
+        for qi in range(Q):
+            for j in range(Hkv * G):
+                h = j // G
+                want = O.dense_attention(O.bf16_bits_to_f64(qb[s, qi, j])[None, :], O.bf16_bits_to_f64(kb[s, h]),
+                                         O.bf16_bits_to_f64(vb[s, h]), L)
+                assert np.abs(out[s, qi, j] - want[0]).max() < 1e-10, (s, qi, j)
+
+
+def test_append_chunk_places_token_c_of_head_h_at_row_length_plus_c():
+    # each row encodes its place: dims 0, 1, 2 hold (sequence, head, token) + 1, exact in bf16
+    B, Hkv, L, C, cap = 2, 3, 5, 4, 12
+    full = np.zeros((B, Hkv, L + C, 128))
+    for s in range(B):
+        for h in range(Hkv):
+            for t in range(L + C):
+                full[s, h, t, :3] = (s + 1, h + 1, t + 1)
+    cache = np.full((B, Hkv, cap, 128), -1.0)
+    cache[:, :, :L] = full[:, :, :L]
+    chunk = np.zeros((B, C, Hkv, 128))  # the chunk's own layout, filled element by element
+    for s in range(B):
+        for c in range(C):
+            for h in range(Hkv):
+                chunk[s, c, h] = full[s, h, L + c]
+    kc, vc = O.append_chunk(_bf16_bits_of(cache), _bf16_bits_of(cache), _bf16_bits_of(chunk),
+                            _bf16_bits_of(chunk), L)
+    assert np.array_equal(O.bf16_bits_to_f64(kc), full)
+    assert np.array_equal(O.bf16_bits_to_f64(vc), full)
+
+
+@pytest.mark.parametrize("L", [0, 37])
+def test_prefill_all_query_i_sees_tokens_below_length_plus_i(L):
+    # k = all: query i of the chunk is dense RoPE attention over tokens [0, L + i) of its
+    # group, at position L + i.  The caches hold garbage past L (only the chunk may fill
+    # it) and the chunk's rows are distinct per (sequence, head, token).
+    B, Hkv, G, C, b = 2, 2, 2, 6, 4
+    rng = np.random.default_rng(23 + L)
+    kf = rng.standard_normal((B, Hkv, L + C, 128))
+    vf = rng.standard_normal((B, Hkv, L + C, 128))
+    kcache = rng.standard_normal((B, Hkv, L + C + 3, 128)) * 50
+    vcache = rng.standard_normal((B, Hkv, L + C + 3, 128)) * 50
+    kcache[:, :, :L], vcache[:, :, :L] = kf[:, :, :L], vf[:, :, :L]
+    knew, vnew = np.zeros((B, C, Hkv, 128)), np.zeros((B, C, Hkv, 128))
+    for s in range(B):
+        for c in range(C):
+            for h in range(Hkv):
+                knew[s, c, h], vnew[s, c, h] = kf[s, h, L + c], vf[s, h, L + c]
+    qb = _bf16_bits_of(rng.standard_normal((B, C, Hkv * G, 128)))
+    out, trees = O.prefill_all(_bf16_bits_of(kcache), _bf16_bits_of(vcache), _bf16_bits_of(knew),
+                               _bf16_bits_of(vnew), qb, np.eye(128), b, L, O.TOPK_ALL)
+    kf, vf = O.round_to_bf16(kf), O.round_to_bf16(vf)
+    for s in range(B):
+        for i in range(C):
+            for j in range(Hkv * G):
+                h = j // G
+                want = O.dense_attention(O.bf16_bits_to_f64(qb[s, i, j])[None, :], kf[s, h, :L + i],
+                                         vf[s, h, :L + i], L + i)
+                assert np.abs(out[s, i, j] - want[0]).max() < 1e-10, (s, i, j)
+    assert trees[0][0].length == L + C
