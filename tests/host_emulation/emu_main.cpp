@@ -156,7 +156,7 @@ int main(int argc, char **argv) {
 
   const int tiles = (int)kv["tiles"], top_k = (int)kv["top_k"], sel_levels = (int)kv["sel_levels"];
   std::vector<float> out(q.size(), 0.f);
-  std::vector<int32_t> sel((size_t)tiles * sel_levels * std::max(top_k, 1), -7), ent((size_t)tiles * 2, 0);
+  std::vector<int32_t> sel((size_t)tiles * sel_levels * std::min(std::max(top_k, 1), 64), -7), ent((size_t)tiles * 2, 0);
 
   AttendArgs a = {};
   a.k_tok = ktok.data();

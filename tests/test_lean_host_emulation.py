@@ -58,12 +58,17 @@ def _rph(G, CS, max_cand):
     raise ValueError("no lean shape")
 
 
-def _run(emu_bin, tmp_path, B, hkv, G, L, b, k, Q, CS, causal=False, seed=1, lens=None):
+def _run(emu_bin, tmp_path, B, hkv, G, L, b, k, Q, CS, causal=False, seed=1, lens=None, zero_keys=False):
     """Lay out the oracle's bf16 tree, run the kernel on host threads, check every tile.
-    lens: per-sequence lengths (decode; L is then their maximum)."""
+    lens: per-sequence lengths (decode; L is then their maximum).  zero_keys: every key
+    is zero, so every score ties at 0 and each level keeps its lowest positions."""
     C = Q if causal else 0
     cap = L + C
     inp = I.random_case(B, L, hkv, hkv * G, Q, seed=seed, capacity=cap, chunk=C)
+    if zero_keys:
+        inp["k_tok"].zero_()
+        if C:
+            inp["k_new"].zero_()
     kb, vb = bits(inp["k_tok"]), bits(inp["v_tok"])
     if causal:
         kb, vb = O.append_chunk(kb, vb, bits(inp["k_new"]), bits(inp["v_new"]), L)
@@ -120,7 +125,7 @@ def _run(emu_bin, tmp_path, B, hkv, G, L, b, k, Q, CS, causal=False, seed=1, len
     assert r.returncode == 0, (r.stdout[-2000:], r.stderr[-4000:])
     assert int(open(d / "err.txt").read()) == 0
     out = np.fromfile(d / "out.bin", np.float32).reshape(B, Q, hkv * G, 128)
-    sel = np.fromfile(d / "sel.bin", np.int32).reshape(tiles, sel_levels, max(k, 1))
+    sel = np.fromfile(d / "sel.bin", np.int32).reshape(tiles, sel_levels, min(max(k, 1), 64))
     ent = np.fromfile(d / "entries.bin", np.int32).reshape(tiles, 2)
 
     qb = bits(inp["q"])
@@ -154,6 +159,7 @@ def test_two_candidates_over_a_cluster(emu_bin, tmp_path, CS):
     (1, 1, 8, 300, 16, 8, 1, 4),    # G = 8 (the only G = 8 shape)
     (1, 1, 4, 700, 8, 0, 2, 4),     # k = 0: the top-level summaries alone
     (2, 1, 4, 4096, 16, 8, 1, 4),   # the 1M tree's per-level shape: 16 -> 128 -> 128 candidates
+    (1, 1, 4, 150, 4, R.TOPK_ALL, 2, 4),  # k = all: every candidate kept, up to 150 a level
 ])
 def test_decode_matches_oracle(emu_bin, tmp_path, B, hkv, G, L, b, k, Q, CS):
     _run(emu_bin, tmp_path, B, hkv, G, L, b, k, Q, CS)
@@ -174,3 +180,10 @@ def test_causal_levels_past_128_candidates(emu_bin, tmp_path):
 def test_decode_with_per_sequence_lengths(emu_bin, tmp_path, CS):
     # an empty sequence, a single token, a shallow tree and the deepest one in one launch
     _run(emu_bin, tmp_path, 4, 1, 4, 1000, 4, 2, 1, CS, lens=[0, 1, 37, 1000], seed=6)
+
+
+@pytest.mark.parametrize("k", [3, 8])
+def test_all_scores_tied_keep_the_lowest_positions(emu_bin, tmp_path, k):
+    # zero keys: every group score is exactly 0, so selection is decided by position alone
+    st = _run(emu_bin, tmp_path, 1, 1, 4, 2000, 8, k, 2, 4, zero_keys=True, seed=7)
+    assert st.near_ties == 0
