@@ -168,16 +168,37 @@ def kernel_source_sha() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(name: str):
-    """DRAM bytes per launch from a committed ncu summary, if it matches the current kernel source."""
+def recorded_profile(name: str):
+    """Numeric fields of a committed ncu summary (profiles/<name>.txt, "key: value" lines),
+    if it was taken on the current kernel source; else None."""
     path = os.path.join(ROOT, "profiles", f"{name}.txt")
     try:
-        kv = dict(line.split(":", 1) for line in open(path) if ":" in line)
-        if kv.get("kernel_source_sha256", "").strip() != kernel_source_sha():
+        kv = {k.strip(): v.strip() for k, v in (line.split(":", 1) for line in open(path) if ":" in line)}
+        if kv.get("kernel_source_sha256", "") != kernel_source_sha():
             return None
-        return float(kv["dram_bytes_per_launch"].strip())
+        out = {}
+        for k, v in kv.items():
+            try:
+                out[k] = float(v)
+            except ValueError:
+                out[k] = v
+        return out
     except Exception:
         return None
+
+
+def recorded_traffic(name: str, tiles: int):
+    """DRAM bytes of a launch of `tiles` tiles from a committed ncu summary of smaller cases
+    (a fixed part per launch plus a part per tile, fitted from two sizes), if it matches the
+    current kernel source."""
+    prof = recorded_profile(name)
+    if prof is None:
+        return None
+    if "fixed_bytes" in prof and "bytes_per_tile" in prof:
+        return prof["fixed_bytes"] + prof["bytes_per_tile"] * tiles
+    if "dram_bytes_per_launch" in prof:
+        return prof["dram_bytes_per_launch"] / prof.get("tiles", tiles) * tiles
+    return None
 
 
 def make_tree(R, p, inp, length, build=True):
@@ -221,17 +242,47 @@ def leg_decode_1m(R, timer, args, dist_on, hbm_peak, peaks_src, heads=None):
     res = dict(per_step_s=per, total_s=total, wall_s=wall, mean_s=mean_s, rows=rows,
                bytes_per_launch=bytes_per_launch, queries=B * Q)
 
-    # end to end through the host-buffer call: pinned host queries in, pinned host output
-    # back, both copies queued by the library inside the timed step
+    # end to end from host buffers, two ways, both inside the timed step: (mapped) the
+    # host-buffer call with pinned buffers, which the kernel reads and writes across the
+    # host link itself; (staged) one copy of the queries to the device, the decode call,
+    # one copy of the output back (pinned buffers, cudaMemcpyAsync each way)
     q_host = q.cpu().pin_memory()
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     q_dev = torch.empty_like(q)
 
-    def e2e_step():
+    def e2e_mapped():
         R.decode_host(p, tree, q_host, out_host, q_dev, out, ws)
 
-    per_e, _ = timer.run(e2e_step, args.steps, args.warmup)
-    res["e2e_total_s"] = max_over_ranks(sum(per_e), dist_on)
+    def e2e_staged():
+        q_dev.copy_(q_host, non_blocking=True)
+        R.decode(p, tree, q_dev, out, ws)
+        out_host.copy_(out, non_blocking=True)
+
+    per_m, _ = timer.run(e2e_mapped, args.steps, args.warmup)
+    per_s, _ = timer.run(e2e_staged, args.steps, args.warmup)
+    t_m = max_over_ranks(sum(per_m), dist_on)
+    t_s = max_over_ranks(sum(per_s), dist_on)
+    # breakdown of the staged step: each piece between its own events, L2 flushed first
+    stream = torch.cuda.current_stream()
+    pieces = {"h2d": [], "kernel": [], "d2h": []}
+    for i in range(max(50, min(args.steps, 400))):
+        timer.flush()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record(stream)
+        q_dev.copy_(q_host, non_blocking=True)
+        ev[1].record(stream)
+        R.decode(p, tree, q_dev, out, ws)
+        ev[2].record(stream)
+        out_host.copy_(out, non_blocking=True)
+        ev[3].record(stream)
+        torch.cuda.synchronize()
+        if i >= 5:
+            for k, (a, b) in zip(pieces, ((0, 1), (1, 2), (2, 3))):
+                pieces[k].append(ev[a].elapsed_time(ev[b]) * 1e3)
+    res["e2e"] = {"mapped_us_per_step": t_m / args.steps * 1e6, "staged_us_per_step": t_s / args.steps * 1e6,
+                  "path": "mapped" if t_m <= t_s else "staged",
+                  "staged_breakdown_us_median": {k: statistics.median(v) for k, v in pieces.items()}}
+    res["e2e_total_s"] = min(t_m, t_s)
     res["h2d"] = q_host.numel() * 2
     res["d2h"] = out_host.numel() * 2
 
@@ -287,13 +338,29 @@ def leg_prefill(R, timer, args, dist_on, hbm_peak, name, length):
     R.check_device_errors(ws)
     del tree, ws, inp
     torch.cuda.empty_cache()
-    return {"workload": f"{name}: B={w.batch}, L={w.length} cached + C={w.chunk} chunk, Hq={w.q_heads}, "
-                        f"Hkv={w.kv_heads}, b={w.branching}, k={w.top_k}",
-            "tokens_per_s": w.batch * w.chunk / t, "ms_per_chunk": t * 1e3,
-            "rows_read": rows, "logical_bytes": logical, "logical_GBps": logical / t / 1e9,
-            "logical_frac_of_hbm": logical / t / 1e9 / hbm_peak,
-            "note": "append + extension build + causal attend per call; rows re-read by neighbouring "
-                    "queries hit L2, so logical GB/s can exceed HBM bandwidth"}
+    res = {"workload": f"{name}: B={w.batch}, L={w.length} cached + C={w.chunk} chunk, Hq={w.q_heads}, "
+                       f"Hkv={w.kv_heads}, b={w.branching}, k={w.top_k}",
+           "tokens_per_s": w.batch * w.chunk / t, "ms_per_chunk": t * 1e3,
+           "rows_read": rows, "logical_bytes": logical, "logical_GBps": logical / t / 1e9,
+           "logical_frac_of_hbm": logical / t / 1e9 / hbm_peak,
+           "note": "append + extension build + causal attend per call; rows re-read by neighbouring "
+                   "queries hit L2, so logical GB/s can exceed HBM bandwidth"}
+    prof = recorded_profile("attend_warp_prefill_counters")
+    if prof is not None:
+        per_tile_dram = prof["dram_bytes_per_launch"] / prof["tiles"]
+        per_tile_inst = prof["warp_inst_per_launch"] / prof["tiles"]
+        dram = per_tile_dram * tiles
+        inst = per_tile_inst * tiles
+        peak_issue = prof["sms"] * 4 * prof["sm_hz"]  # one warp instruction per sub-partition per cycle
+        res["dram"] = {"bytes_per_chunk": dram, "GBps": dram / t / 1e9, "frac_of_hbm": dram / t / 1e9 / hbm_peak,
+                       "time": "the whole chunk call (append + extension + attend)",
+                       "source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the attend kernel on the "
+                                 f"{prof['case']} case, per tile, times this call's {tiles} tiles"}
+        res["issue"] = {"warp_inst_per_chunk": inst, "frac_of_peak_issue": inst / t / peak_issue,
+                        "peak_issue_per_s": peak_issue,
+                        "source": "ncu smsp__inst_executed.sum of the attend kernel on the same case, per tile; "
+                                  "peak = SMs x 4 sub-partitions x SM clock"}
+    return res
 
 
 def leg_decode_loop(R, timer, args, dist_on):
@@ -483,6 +550,130 @@ def leg_build_2m(R, timer, args, dist_on, hbm_peak):
 
 # ----------------------------------------------------------------------------- oracle (CPU baseline)
 
+class _NoBarrier:
+    def wait(self):
+        pass
+
+
+_WORKER_BARRIER = None
+
+
+def _oracle_pool_init(barrier):
+    global _WORKER_BARRIER
+    _WORKER_BARRIER = barrier
+
+
+def oracle_sample(kind: str, budget_s: float, seed: int) -> dict:
+    """One host worker of the oracle baseline: builds its own bounded sample of a workload
+    (untimed), waits for the other workers, then times the oracle on it.
+
+      decode:  one KV group of the decode_1m recipe (L = 2^20, b = 16, k = 8); tiles are
+               decode queries of that group (the first from the recipe, the rest seeded
+               N(0, 1) queries); a decode query of the workload is 8 tiles.
+      prefill: one KV group of the prefill_524k recipe (L = 524288 cached + C = 8192), tree
+               built over L + C; tiles are causal queries at p = L + i, i drawn from the
+               chunk; a prefill token is 8 tiles.  The append and tree extension are not
+               timed (the tree is built untimed).
+      build:   recsa_build over one KV head of 2^18 tokens of the build_decode_2m recipe,
+               repeated; bytes = token rows read + node rows written (K and V)."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    from oracle import recsa_oracle as O
+
+    barrier = _WORKER_BARRIER or _NoBarrier()
+    with threadpool_limits(limits=1):
+        if kind == "decode":
+            w = dataclasses.replace(I.WORKLOADS["decode_1m"], batch=1, kv_heads=1, q_heads=4)
+            inp = I.decode_inputs(w, device="cpu")
+            tree = O.build_tree(O.bf16_bits_to_f64(I.bf16_bits(inp["k_tok"][0, 0])),
+                                O.bf16_bits_to_f64(I.bf16_bits(inp["v_tok"][0, 0])), inp["pooler"].double().numpy(),
+                                w.branching)
+            q0 = O.bf16_bits_to_f64(I.bf16_bits(inp["q"][0, 0]))
+            del inp
+            rng = np.random.default_rng(seed)
+            barrier.wait()
+            tiles, t0 = 0, time.perf_counter()
+            while True:
+                O.attend(q0 if tiles == 0 else rng.standard_normal((4, 128)), tree, w.length, w.top_k)
+                tiles += 1
+                el = time.perf_counter() - t0
+                if el >= budget_s:
+                    break
+            return {"units": tiles, "seconds": el}
+        if kind == "prefill":
+            w = dataclasses.replace(I.WORKLOADS["prefill_524k"], kv_heads=1, q_heads=4)
+            inp = I.prefill_inputs(w, device="cpu")
+            kb, vb = I.bf16_bits(inp["k_tok"][0, 0, :w.length]), I.bf16_bits(inp["v_tok"][0, 0, :w.length])
+            kt = np.concatenate([O.bf16_bits_to_f64(kb), O.bf16_bits_to_f64(I.bf16_bits(inp["k_new"][0, :, 0]))])
+            vt = np.concatenate([O.bf16_bits_to_f64(vb), O.bf16_bits_to_f64(I.bf16_bits(inp["v_new"][0, :, 0]))])
+            tree = O.build_tree(kt, vt, inp["pooler"].double().numpy(), w.branching)
+            qb = I.bf16_bits(inp["q"][0])
+            del inp, kt, vt
+            rng = np.random.default_rng(seed)
+            barrier.wait()
+            tiles, t0 = 0, time.perf_counter()
+            while True:
+                i = int(rng.integers(0, w.chunk))
+                O.attend(O.bf16_bits_to_f64(qb[i]), tree, w.length + i, w.top_k, causal=True)
+                tiles += 1
+                el = time.perf_counter() - t0
+                if el >= budget_s:
+                    break
+            return {"units": tiles, "seconds": el}
+        if kind == "build":
+            w = dataclasses.replace(I.WORKLOADS["build_decode_2m"], length=1 << 18, kv_heads=1, q_heads=4)
+            inp = I.decode_inputs(w, device="cpu")
+            kt = O.bf16_bits_to_f64(I.bf16_bits(inp["k_tok"][0, 0]))
+            vt = O.bf16_bits_to_f64(I.bf16_bits(inp["v_tok"][0, 0]))
+            W = inp["pooler"].double().numpy()
+            del inp
+            nodes = sum(O.level_counts(w.length, w.branching)[1:])
+            per_build = (w.length + nodes) * 2 * ROW  # K and V: every token row read, every node row written
+            barrier.wait()
+            builds, t0 = 0, time.perf_counter()
+            while True:
+                O.build_tree(kt, vt, W, w.branching)
+                builds += 1
+                el = time.perf_counter() - t0
+                if el >= budget_s:
+                    break
+            return {"units": builds, "seconds": el, "bytes_per_unit": per_build}
+    raise ValueError(kind)
+
+
+def oracle_workers_for_ram() -> int:
+    """Host workers for the all-core oracle figures: every core, at most one worker per
+    5 GB of available memory (a worker holds one fp64 tree of ~2-3 GB)."""
+    import psutil
+
+    cores = os.cpu_count() or 1
+    avail = psutil.virtual_memory().available / 2 ** 30
+    return max(1, min(cores, int((avail - 8) // 5), 64))
+
+
+def oracle_baseline(budget_s: float) -> dict:
+    """The fp64 oracle on the host cores: decode, prefill and build, each on one core and on
+    `workers` spawned processes (one core each, numpy limited to one thread) that build
+    their samples first and start timing together."""
+    import multiprocessing as mp
+
+    workers = oracle_workers_for_ram()
+    out = {"cores_available": os.cpu_count(), "workers": workers}
+    for kind in ("decode", "prefill", "build"):
+        one = oracle_sample(kind, budget_s, seed=1)
+        res = {"cores_1": one}
+        if workers > 1:
+            ctx = mp.get_context("spawn")
+            barrier = ctx.Barrier(workers)
+            with ctx.Pool(workers, initializer=_oracle_pool_init, initargs=(barrier,)) as pool:
+                parts = pool.starmap(oracle_sample, [(kind, budget_s, 100 + i) for i in range(workers)])
+            res["cores_all"] = {"units": sum(x["units"] for x in parts), "seconds": max(x["seconds"] for x in parts),
+                                "bytes_per_unit": parts[0].get("bytes_per_unit")}
+        out[kind] = res
+    return out
+
+
 def oracle_decode_rate(budget_s: float, device_inputs=None, max_tiles=None, warmup_tiles=0):
     """The fp64 oracle's decode rate on a bounded sample of the 1M workload.
 
@@ -564,15 +755,17 @@ def run_reference(args):
 
 
 def run_profile_case(args):
-    """Small case of one kernel for an ncu capture (a few launches, about 1 GB on the device).
+    """Small case of one kernel for an ncu capture (a few launches, a few GB on the device).
 
     decode: the 1M-context decode tile structure of the headline (b = 16, k = 8, needles)
-    with 1 sequence and 2 KV groups (2 tiles per launch instead of 32)."""
+    with 1 sequence and --profile-kv-heads KV groups (2 by default: 2 tiles per launch
+    instead of 32, about 1 GB of caches)."""
     import hierarchical_sparse_attention_build_b200 as R
 
     torch.cuda.set_device(0)
     if args.profile == "decode":
-        w = dataclasses.replace(I.WORKLOADS["decode_1m"], batch=1, kv_heads=2, q_heads=8)
+        kvh = args.profile_kv_heads
+        w = dataclasses.replace(I.WORKLOADS["decode_1m"], batch=1, kv_heads=kvh, q_heads=4 * kvh)
         inp = I.decode_inputs(w, device="cuda")
         p = R.params(num_kv_heads=w.kv_heads, num_q_heads=w.q_heads, branching=w.branching, top_k=w.top_k)
         tree, ws = make_tree(R, p, inp, w.length)
@@ -672,11 +865,35 @@ def run_gpu(args):
     clk = clocks.stop()
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        r = oracle_decode_rate(budget_s=args.cpu_seconds)
-        cpu = {"value": r["queries_per_s"], "unit": "queries/s", "cores": 1, "kind": "oracle",
-               "sample": f"{r['tiles']} query-group tiles in {r['seconds']:.1f} s over the trees of 2 KV heads of "
-                         f"{r['source']} (trees built untimed, {r['tree_build_s']:.1f} s); queries/s = tiles/s / 8; "
-                         "numpy limited to 1 thread"}
+        ob = oracle_baseline(args.cpu_seconds)
+
+        def rate(r, div=1.0):
+            return None if r is None else r["units"] / r["seconds"] / div
+
+        dec1, decn = ob["decode"]["cores_1"], ob["decode"].get("cores_all")
+        pre1, pren = ob["prefill"]["cores_1"], ob["prefill"].get("cores_all")
+        bld1, bldn = ob["build"]["cores_1"], ob["build"].get("cores_all")
+        nw = ob["workers"]
+        best = decn if decn is not None else dec1
+        cpu = {"value": rate(best, 8.0), "unit": "queries/s", "cores": nw if decn is not None else 1,
+               "kind": "oracle",
+               "sample": f"decode_1m recipe, one KV group per worker (tree of 2^20 tokens built untimed), "
+                         f"{best['units']} query-group tiles in {best['seconds']:.1f} s on {nw if decn else 1} worker "
+                         "process(es), one core each (numpy limited to 1 thread); queries/s = tiles/s / 8 "
+                         "(8 KV groups a query)",
+               "cores_available": ob["cores_available"],
+               "decode_queries_per_s": {"cores_1": rate(dec1, 8.0), "cores_all": rate(decn, 8.0)},
+               "prefill_tokens_per_s": {"cores_1": rate(pre1, 8.0), "cores_all": rate(pren, 8.0),
+                                        "sample": "prefill_524k recipe, one KV group per worker (tree over "
+                                                  "524288 + 8192 tokens built untimed); causal attend of random "
+                                                  "chunk queries; tokens/s = tiles/s / 8; the append and tree "
+                                                  "extension are not timed"},
+               "build_GBps": {"cores_1": None if bld1 is None else bld1["units"] * bld1["bytes_per_unit"] / bld1["seconds"] / 1e9,
+                              "cores_all": None if bldn is None else bldn["units"] * bldn["bytes_per_unit"] / bldn["seconds"] / 1e9,
+                              "sample": "build of one KV head of 2^18 tokens (b = 16) per worker, repeated; bytes = "
+                                        "token rows read + node rows written, K and V"},
+               "workers_note": "all-core figures: one spawned process per core, at most one per 5 GB of free "
+                               "host memory"}
     if dist_on:
         import torch.distributed as dist
         dist.barrier()
@@ -693,7 +910,7 @@ def run_gpu(args):
     w_all = I.WORKLOADS["decode_1m"]
     mean_s = dec["mean_s"]
     achieved = dec["bytes_per_launch"] / mean_s / 1e9
-    traffic = recorded_traffic("decode_1m_attend_traffic")
+    traffic = recorded_traffic("decode_1m_attend_traffic", B * w.kv_heads)
     line = {
         "metric": METRIC,
         "value": value,
@@ -720,7 +937,7 @@ def run_gpu(args):
                      "algorithmic_bytes_per_launch": dec["bytes_per_launch"],
                      "peak_source": f"{peaks_src} hbm_gbs (MEASURED_PEAKS.json)"},
         "e2e": {"value": job_queries * args.steps / dec["e2e_total_s"], "unit": "queries/s",
-                "h2d_bytes_per_step": dec["h2d"], "d2h_bytes_per_step": dec["d2h"]},
+                "h2d_bytes_per_step": dec["h2d"], "d2h_bytes_per_step": dec["d2h"], **dec["e2e"]},
         "gpu_launches": args.steps,
         "clocks": clk,
         "decode": {"us_per_step_median": statistics.median(dec["per_step_s"]) * 1e6,
@@ -742,11 +959,13 @@ def main():
     ap.add_argument("--quick", action="store_true", help="fewer sweep points and steps in the side legs")
     ap.add_argument("--headline-only", action="store_true", help="skip the prefill and build legs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-seconds", type=float, default=6.0)
     ap.add_argument("--shard", default="sequences", choices=["sequences", "heads"],
                     help="with N GPUs: N replicas of the batch (sequences, weak scaling) or the batch's "
                          "KV heads split over the N GPUs (heads, strong scaling)")
     ap.add_argument("--profile", choices=["decode", "prefill", "build", "append", "decode_loop"], help="run a small case of one kernel for ncu")
+    ap.add_argument("--profile-kv-heads", type=int, default=2,
+                    help="--profile decode: KV heads of the one 1M-token sequence (tiles per launch)")
     args = ap.parse_args()
     if args.profile:
         run_profile_case(args)

@@ -508,9 +508,12 @@ RECSA_API recsa_status recsa_check_device_errors(void *ws, recsa_stream_t stream
   if (!ws) return fail(RECSA_ERR_INVALID_ARGUMENT, "workspace is NULL");
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail((int)e, "synchronize");
-  uint32_t word = 0;
+  uint32_t word = 0, build_word = 0;
   e = cudaMemcpy(&word, ws, sizeof word, cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail((int)e, "read error word");
+  const int rc = read_build_errors(&build_word);  // the build kernels' word (they take no workspace)
+  if (rc != 0) return cuda_fail(rc, "read the build error word");
+  word |= build_word;
   if (word == 0) return RECSA_OK;
   const uint32_t zero = 0;
   e = cudaMemcpy(ws, &zero, sizeof zero, cudaMemcpyHostToDevice);

@@ -13,19 +13,16 @@
 
 #include "recsa_device.cuh"
 #include "recsa_internal.h"
+#include "recsa_umma.cuh"
 
 namespace recsa {
+
+// Set by a build or append kernel whose wait on the tensor cores gave up (reported by
+// recsa_check_device_errors); the kernel leaves the affected keys unwritten and returns.
+__device__ uint32_t g_build_err;
+
 namespace {
 
-constexpr int kBuildThreads = 256;
-constexpr int kBuildWarps = kBuildThreads / 32;
-// Nodes per warp: 8 for a whole level; 1 for small launches (a prefill or decode step
-// extends one node per level and head), so their nodes run side by side, not in turn.
-constexpr int kNodesPerWarp = 8;
-constexpr int kFewNodes = 1;
-__host__ __device__ constexpr size_t build_smem(int npw) {
-  return (size_t)(kD * kD + kBuildWarps * npw * kD) * sizeof(float);
-}
 
 struct BuildArgs {
   const uint16_t *src_k;  // level l-1 rows (token cache or node arena)
@@ -69,30 +66,6 @@ struct PagedRows {
     return (int64_t)pg * stride + (c & ((int64_t(1) << shift) - 1));
   }
 };
-
-// Wt[k][o] = W[o][k] into shared memory.  A thread moves 16-byte pieces of W; the 32 lanes of
-// a warp take 32 consecutive rows o at the same column, so each shared-memory store fills 32
-// banks, and a thread's pieces are all loaded before any is stored.
-template <int NT>
-__device__ __forceinline__ void load_wt(const float *__restrict__ W, float *Wt, int tid) {
-  constexpr int kPieces = kD * kD / 4 / NT;
-  static_assert(kD * kD / 4 % NT == 0, "threads must divide the pooler's 16-byte pieces");
-  float4 w[kPieces];
-#pragma unroll
-  for (int i = 0; i < kPieces; ++i) {
-    const int e = tid + i * NT;  // piece e: row o = e % 128, columns 4 * (e / 128) .. +3
-    w[i] = __ldg(reinterpret_cast<const float4 *>(W) + (e & (kD - 1)) * (kD / 4) + (e >> 7));
-  }
-#pragma unroll
-  for (int i = 0; i < kPieces; ++i) {
-    const int e = tid + i * NT;
-    const int o = e & (kD - 1), k = (e >> 7) * 4;
-    Wt[(k + 0) * kD + o] = w[i].x;
-    Wt[(k + 1) * kD + o] = w[i].y;
-    Wt[(k + 2) * kD + o] = w[i].z;
-    Wt[(k + 3) * kD + o] = w[i].w;
-  }
-}
 
 // One child row piece (the lane's 4 dims): through the read-only path for a level written by
 // an earlier launch, an ordinary load for one this kernel may have written.
@@ -150,46 +123,6 @@ __device__ __forceinline__ void node_means(const uint16_t *kb, const uint16_t *v
   }
 }
 
-// key = W @ mean for NPW nodes whose key means are rows [NPW][128] in shared memory; lane
-// owns outputs 4*lane .. 4*lane+3, as the pairs (4l, 4l+1) and (4l+2, 4l+3) of packed fp32
-// FMAs (each output's terms in k order).
-template <int NPW>
-__device__ __forceinline__ void apply_w(const float *Wt, const float *mean_rows, int lane, float acc[NPW][4]) {
-  float2 acc2[NPW][2];
-#pragma unroll
-  for (int n = 0; n < NPW; ++n) acc2[n][0] = acc2[n][1] = make_float2(0.f, 0.f);
-  const float4 *Wt4 = reinterpret_cast<const float4 *>(Wt);
-  const float4 *M4 = reinterpret_cast<const float4 *>(mean_rows);
-#pragma unroll 2
-  for (int k = 0; k < kD; k += 4) {
-    float2 w[4][2];
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const float4 wt = Wt4[(k + t) * 32 + lane];
-      w[t][0] = make_float2(wt.x, wt.y);
-      w[t][1] = make_float2(wt.z, wt.w);
-    }
-#pragma unroll
-    for (int n = 0; n < NPW; ++n) {
-      const float4 m = M4[n * 32 + (k >> 2)];
-      const float mt[4] = {m.x, m.y, m.z, m.w};
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const float2 mm = make_float2(mt[t], mt[t]);
-        acc2[n][0] = __ffma2_rn(mm, w[t][0], acc2[n][0]);
-        acc2[n][1] = __ffma2_rn(mm, w[t][1], acc2[n][1]);
-      }
-    }
-  }
-#pragma unroll
-  for (int n = 0; n < NPW; ++n) {
-    acc[n][0] = acc2[n][0].x;
-    acc[n][1] = acc2[n][0].y;
-    acc[n][2] = acc2[n][1].x;
-    acc[n][3] = acc2[n][1].y;
-  }
-}
-
 __device__ __forceinline__ void store_row4(uint16_t *p, const float x[4]) {
   uint2 o;
   o.x = pack_bf16x2(x[0], x[1]);
@@ -197,72 +130,168 @@ __device__ __forceinline__ void store_row4(uint16_t *p, const float x[4]) {
   *reinterpret_cast<uint2 *>(p) = o;
 }
 
-// One CTA handles blocks of 8 * NPW nodes: each warp streams the children of NPW nodes
-// (lane = 4 consecutive dims, one 256-byte row per warp load), forms the child means in
-// fp32, writes the value rows, then applies W to its own key means (W^T resident in shared
-// memory).  Warps share only W^T, so they never wait for one another after it is loaded.
-template <int NPW, bool kPaged>
-__global__ void __launch_bounds__(kBuildThreads, 2) build_level_kernel(const BuildArgs a) {
-  constexpr int kNodesPerBlock = kBuildWarps * NPW;
-  extern __shared__ __align__(16) float smem_f[];
-  float *Wt = smem_f;               // Wt[k][o] = W[o][k]
-  float *Mean = smem_f + kD * kD;   // [8 * NPW][128] key means
+// The level build with the pooler product on the tensor cores.  One CTA per SM, persistent
+// over tiles of 128 nodes (the level's nodes of every (sequence, head), in order).  Warp w
+// streams nodes 8w .. 8w+7 of a tile: the children's sums give the value row (stored at
+// once) and the key mean, whose three bf16 parts go to row 8w + n of the A operand.  Then
+// one thread issues the pooler product into one of two TMEM accumulators (W, the B operand,
+// stays in shared memory), and the warps stream the next tile while the tensor cores work.
+// The finished accumulator is read back during the next tile (warp w: lanes 32 (w % 4) ..,
+// columns 32 (w / 4) ..), rounded to bf16 and stored.  A is single-buffered: a tile's first
+// A row is written once the previous tile's product has completed.  Sixteen warps keep 16
+// nodes' children (128 KB) in flight per SM.
+constexpr int kMmaThreads = 512;
+constexpr int kMmaWarps = kMmaThreads / 32;
+constexpr int kMmaNodesPerWarp = umma::kM / kMmaWarps;  // 16
+constexpr size_t kMmaSmem = 2 * (size_t)umma::kOperandBytes + 128;  // A, B, barriers, TMEM address
+
+template <bool kPaged>
+__global__ void __launch_bounds__(kMmaThreads, 1) build_level_mma_kernel(const BuildArgs a) {
+  extern __shared__ __align__(128) unsigned char smem_u8[];
+  unsigned char *A = smem_u8, *Bop = smem_u8 + umma::kOperandBytes;
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem_u8 + 2 * umma::kOperandBytes);  // product done, by accumulator
+  uint32_t *tmem_s = reinterpret_cast<uint32_t *>(bar + 2);
+  uint32_t *flag_s = tmem_s + 1;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  load_wt<kBuildThreads>(a.pooler, Wt, tid);
+  if (warp == 0) {
+    umma::tmem_alloc(tmem_s, 2 * umma::kTmemCols);
+    umma::tmem_relinquish();
+  }
+  if (tid == 32) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    mbar_fence_init();
+    *flag_s = 0u;
+  }
+  umma::load_pooler_operand<kMmaThreads>(a.pooler, Bop, tid);
+  umma::fence_async_smem();
+  umma::fence_before_sync();
   __syncthreads();
+  umma::fence_after_sync();
+  const uint32_t tmem = *tmem_s;
 
   const int64_t total = (int64_t)a.bh * a.nj;
-  for (int64_t base = (int64_t)blockIdx.x * kNodesPerBlock; base < total;
-       base += (int64_t)gridDim.x * kNodesPerBlock) {
-    bool live[NPW];
-    for (int t = 0; t < NPW; ++t) {
-      const int nl = warp * NPW + t;
-      const int64_t id = base + nl;
-      float ks[4] = {0.f, 0.f, 0.f, 0.f}, vs[4] = {0.f, 0.f, 0.f, 0.f};
-      live[t] = id < total;
-      if (live[t]) {
-        const int64_t bhi = id / a.nj;
-        const int64_t j = a.j0 + id % a.nj;
-        int64_t length = a.length, n_prev = a.n_prev;
-        if (a.seq_len) {  // this sequence's own length: its level has ceil(len / b^l) nodes
-          length = min(max(a.seq_len[bhi / a.hkv], (int64_t)0), a.length);
-          n_prev = (length + a.span_prev - 1) / a.span_prev;
-          live[t] = j < (length + a.span - 1) / a.span;
-        }
-        if (live[t]) {
-          const int64_t c0 = j * a.b;
-          const int64_t c1 = min(c0 + (int64_t)a.b, n_prev);
-          if (kPaged) {  // level 1 over a paged token cache
-            const int64_t h = bhi % a.hkv;
-            const PagedRows rows{a.pages + (bhi / a.hkv) * a.pages_per_seq, (int64_t)a.hkv << a.page_shift,
-                                 a.page_shift, a.num_pages};
-            const uint16_t *kb = a.src_k + (h << a.page_shift) * kD + lane * 4;
-            const uint16_t *vb = a.src_v + (h << a.page_shift) * kD + lane * 4;
-            node_means<true>(kb, vb, c0, c1, n_prev, length, a.span_prev, ks, vs, rows);
-          } else {
-            const uint16_t *kb = a.src_k + (a.src_row_off + bhi * a.src_slots) * kD + lane * 4;
-            const uint16_t *vb = a.src_v + (a.src_row_off + bhi * a.src_slots) * kD + lane * 4;
-            node_means<true>(kb, vb, c0, c1, n_prev, length, a.span_prev, ks, vs, PlainRows{});
-          }
-          store_row4(a.dst_v + (a.dst_row_off + bhi * a.dst_slots + j) * kD + lane * 4, vs);
-        }
-      }
-      *reinterpret_cast<float4 *>(Mean + nl * kD + lane * 4) = make_float4(ks[0], ks[1], ks[2], ks[3]);
+  const int64_t tiles = (total + umma::kM - 1) / umma::kM;
+  // node `id` of the launch: (sequence, head), node index, and whether it exists at its
+  // sequence's length
+  auto locate = [&](int64_t id, int64_t &bhi, int64_t &j, int64_t &length, int64_t &n_prev) -> bool {
+    if (id >= total) return false;
+    bhi = id / a.nj;
+    j = a.j0 + id % a.nj;
+    length = a.length;
+    n_prev = a.n_prev;
+    if (a.seq_len) {  // this sequence's own length: its level has ceil(len / b^l) nodes
+      length = min(max(a.seq_len[bhi / a.hkv], (int64_t)0), a.length);
+      n_prev = (length + a.span_prev - 1) / a.span_prev;
+      return j < (length + a.span - 1) / a.span;
     }
-    __syncwarp();  // a warp applies W to its own nodes only: warps run out of step, so some
-                   // stream children while others compute
-    float acc[NPW][4];
-    apply_w<NPW>(Wt, Mean + warp * NPW * kD, lane, acc);
+    return true;
+  };
+  // the accumulator of tile `tile` (buffer buf) -> key rows
+  auto epilogue = [&](int64_t tile, int buf) {
+    const int rq = warp & 3, cq = warp >> 2;  // lanes 32 rq .., columns 32 cq ..
+    const int row = 32 * rq + lane;
+    uint32_t v[32];
+    umma::tmem_ld32(tmem + (uint32_t)buf * umma::kTmemCols + ((uint32_t)(32 * rq) << 16) + 32u * cq, v);
+    umma::tmem_wait_ld();
+    int64_t bhi, j, length, n_prev;
+    if (locate(tile * umma::kM + row, bhi, j, length, n_prev)) {
+      uint4 *dst = reinterpret_cast<uint4 *>(a.dst_k + (a.dst_row_off + bhi * a.dst_slots + j) * kD + 32 * cq);
 #pragma unroll
-    for (int n = 0; n < NPW; ++n) {
-      const int64_t id = base + warp * NPW + n;
-      if (live[n]) {
-        const int64_t bhi = id / a.nj;
-        const int64_t j = a.j0 + id % a.nj;
-        store_row4(a.dst_k + (a.dst_row_off + bhi * a.dst_slots + j) * kD + lane * 4, acc[n]);
-      }
+      for (int q = 0; q < 4; ++q)
+        dst[q] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
+                            pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                            pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                            pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
     }
-    __syncwarp();  // this warp's Mean rows are rewritten next
+  };
+
+  uint32_t ph[2] = {0u, 0u};
+  bool pending[2] = {false, false};  // a product issued on the accumulator and not yet waited for
+  bool ok = true;
+  int64_t prev = -1;
+  int it = 0;
+  for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++it) {
+    const int buf = it & 1;
+    for (int n = 0; n < kMmaNodesPerWarp; ++n) {
+      const int row = warp * kMmaNodesPerWarp + n;
+      int64_t bhi, j, length, n_prev;
+      float ks[4] = {0.f, 0.f, 0.f, 0.f}, vs[4] = {0.f, 0.f, 0.f, 0.f};
+      if (locate(tile * umma::kM + row, bhi, j, length, n_prev)) {
+        const int64_t c0 = j * a.b;
+        const int64_t c1 = min(c0 + (int64_t)a.b, n_prev);
+        if (kPaged) {  // level 1 over a paged token cache
+          const int64_t h = bhi % a.hkv;
+          const PagedRows rows{a.pages + (bhi / a.hkv) * a.pages_per_seq, (int64_t)a.hkv << a.page_shift,
+                               a.page_shift, a.num_pages};
+          const uint16_t *kb = a.src_k + (h << a.page_shift) * kD + lane * 4;
+          const uint16_t *vb = a.src_v + (h << a.page_shift) * kD + lane * 4;
+          node_means<true>(kb, vb, c0, c1, n_prev, length, a.span_prev, ks, vs, rows);
+        } else {
+          const uint16_t *kb = a.src_k + (a.src_row_off + bhi * a.src_slots) * kD + lane * 4;
+          const uint16_t *vb = a.src_v + (a.src_row_off + bhi * a.src_slots) * kD + lane * 4;
+          node_means<true>(kb, vb, c0, c1, n_prev, length, a.span_prev, ks, vs, PlainRows{});
+        }
+        store_row4(a.dst_v + (a.dst_row_off + bhi * a.dst_slots + j) * kD + lane * 4, vs);
+      }
+      if (n == 0 && prev >= 0) {
+        // the previous tile's product has read A: its accumulator is read back below
+        const int pb = buf ^ 1;
+        const bool done = __all_sync(0xffffffffu, mbar_wait(&bar[pb], ph[pb]));  // one answer a warp
+        if (!done) {
+          ok = false;
+          break;
+        }
+        ph[pb] ^= 1u;
+        pending[pb] = false;
+        umma::fence_after_sync();
+      }
+      umma::store_row4_parts(A, row, lane * 4, ks);
+    }
+    if (!ok && lane == 0) atomicOr(flag_s, 1u);
+    __syncthreads();
+    if (*flag_s) {
+      ok = false;
+      break;
+    }
+    if (prev >= 0) epilogue(prev, buf ^ 1);
+    // every row of A written: visible to the tensor cores, then one thread issues the product
+    umma::fence_async_smem();
+    umma::fence_before_sync();
+    __syncthreads();
+    if (tid == 0) {
+      umma::fence_after_sync();
+      umma::issue_pooler(tmem + (uint32_t)buf * umma::kTmemCols, smem_u32(A), smem_u32(Bop));
+      umma::commit(&bar[buf]);
+    }
+    pending[buf] = true;
+    prev = tile;
+  }
+  if (ok && prev >= 0) {
+    const int pb = (it - 1) & 1;
+    if (__all_sync(0xffffffffu, mbar_wait(&bar[pb], ph[pb]))) {
+      ph[pb] ^= 1u;
+      pending[pb] = false;
+      umma::fence_after_sync();
+      epilogue(prev, pb);
+    } else {
+      ok = false;
+    }
+  }
+  if (!ok && lane == 0) atomicOr(flag_s, 1u);
+  __syncthreads();
+  if (*flag_s && tid == 0) {
+    // a product did not complete within the wait limit: report it, and give the tensor
+    // cores a last bounded wait on every product still out before the accumulators are freed
+    atomicOr(&g_build_err, kErrTimeout);
+    for (int b2 = 0; b2 < 2; ++b2)
+      if (pending[b2]) mbar_wait(&bar[b2], ph[b2]);
+  }
+  umma::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    umma::fence_after_sync();
+    umma::tmem_dealloc(tmem, 2 * umma::kTmemCols);
   }
 }
 
@@ -271,12 +300,11 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_level_kernel(const Bui
 // each level l, the nodes [j0[l], j1[l]) whose spans meet the new tokens (the nodes above
 // them are those nodes' ancestors).  A thread owns one dimension of the key (threads
 // 0..127) or of the value (128..255): it sums that dimension over the node's children and
-// forms its mean.  The key output o = W[o] . mean is one fp32 FMA chain over k = 0..127: the
-// key thread of dimension o runs k < 64 and the value thread of the same o continues with
-// k >= 64, each with its half of W row o in registers.  Per element these are the level
-// build's operations in the level build's order, so the extended tree equals a full build
-// bit for bit.  Rows written at level l are read at level l+1 by other threads of the same
-// CTA after a __syncthreads; no two CTAs touch the same rows.
+// forms its mean, in the level build's operation order.  The level's key means (up to 128
+// nodes at a time) go to the A operand and one thread issues the same split-bf16 pooler
+// product as the level build, so the extended tree equals a full build bit for bit.  Rows
+// written at level l are read at level l+1 by other threads of the same CTA after a
+// __syncthreads; no two CTAs touch the same rows.
 struct ExtendArgs {
   const uint4 *k_new, *v_new;   // [B][C][Hkv][128] bf16, as 16-byte pieces
   uint16_t *k_tok, *v_tok;      // [B][Hkv][capacity][128]
@@ -294,12 +322,9 @@ struct ExtendArgs {
   int64_t span[kMaxLevels + 1];
 };
 constexpr int kExtendThreads = 2 * kD;  // one thread per key dimension and per value dimension
-constexpr int kHalfK = kD / 2;          // W columns held by each thread of a dimension
-// W^T staged as Wt[k][o ^ (k / 4 % 32)]: the coalesced row loads (a warp reads one W row)
-// and the per-thread row reads both hit 32 distinct banks.
-// W^T staging, the key mean, the first half of the key, and per level the rebuilt node range
-// [j0, j1) and the node count of the level below
-constexpr size_t kExtendSmem = (size_t)(kD * kD + 2 * kD) * sizeof(float) + 3 * (kMaxLevels + 1) * sizeof(int64_t);
+// the A and B operands of the pooler product, the product's barrier and the TMEM address, and
+// per level the rebuilt node range [j0, j1) and the node count of the level below
+constexpr size_t kExtendSmem = 2 * (size_t)umma::kOperandBytes + 128 + 3 * (kMaxLevels + 1) * sizeof(int64_t);
 
 // x / y and ceil(x / y) for x >= 0, y >= 1, in 32 bits whenever the operands fit (a 64-bit
 // division is a long instruction sequence; lengths and spans of real trees fit 32 bits).
@@ -316,12 +341,12 @@ __device__ __forceinline__ void prefetch_l2(const void *p) {
 
 template <bool kPaged>
 __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendArgs a) {
-  extern __shared__ __align__(16) float smem_f[];
-  float *Wt = smem_f;               // swizzled W^T (staging only)
-  float *mean = smem_f + kD * kD;   // the node's key mean
-  float *part = mean + kD;          // key outputs after k < 64
-  int64_t *lv_j0 = reinterpret_cast<int64_t *>(part + kD);  // per level: nodes [j0, j1) rebuilt,
-  int64_t *lv_j1 = lv_j0 + (kMaxLevels + 1);                 // the level below's node count
+  extern __shared__ __align__(128) unsigned char smem_u8[];
+  unsigned char *A = smem_u8, *Bop = smem_u8 + umma::kOperandBytes;
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem_u8 + 2 * umma::kOperandBytes);
+  uint32_t *tmem_s = reinterpret_cast<uint32_t *>(bar + 1);
+  int64_t *lv_j0 = reinterpret_cast<int64_t *>(smem_u8 + 2 * umma::kOperandBytes + 128);  // per level: nodes
+  int64_t *lv_j1 = lv_j0 + (kMaxLevels + 1);  // [j0, j1) rebuilt, the level below's node count
   int64_t *lv_np = lv_j1 + (kMaxLevels + 1);
   const int tid = threadIdx.x;
   const int64_t bhi = blockIdx.x;   // (sequence, head)
@@ -356,12 +381,16 @@ __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendA
                         (int64_t)a.hkv << a.page_shift, a.page_shift, a.num_pages};
   auto tok_row = [&](int64_t t) -> int64_t { return kPaged ? paged(t) : t; };
 
-  // W in flight (a warp reads one 512-byte row) while the tokens are appended and the first
-  // children load
-  constexpr int kPieces = kD * kD / 4 / kExtendThreads;
-  float4 w[kPieces];
-#pragma unroll
-  for (int i = 0; i < kPieces; ++i) w[i] = __ldg(reinterpret_cast<const float4 *>(a.pooler) + tid + i * kExtendThreads);
+  const int warp = tid >> 5, lane = tid & 31;
+  if (warp == 0) {
+    umma::tmem_alloc(tmem_s, umma::kTmemCols);
+    umma::tmem_relinquish();
+  }
+  if (tid == 32) {
+    mbar_init(bar, 1);
+    mbar_fence_init();
+  }
+  umma::load_pooler_operand<kExtendThreads>(a.pooler, Bop, tid);  // W, the B operand, in its three parts
   {
     const int64_t s = bhi / a.hkv;
     for (int64_t e = tid; e < (int64_t)a.chunk * 16; e += kExtendThreads) {  // 16 pieces a row
@@ -373,7 +402,14 @@ __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendA
       reinterpret_cast<uint4 *>(a.v_tok)[dst] = __ldg(a.v_new + src);
     }
   }
-  __syncthreads();  // the level ranges are in place, and the appended rows are read below by other threads
+  umma::fence_async_smem();
+  umma::fence_before_sync();
+  __syncthreads();  // the level ranges, W and the TMEM address are in place, and the appended rows are
+                    // read below by other threads
+  umma::fence_after_sync();
+  const uint32_t tmem = *tmem_s;
+  uint32_t ph = 0u;
+  bool ok = true;
   // every child row the walk reads above level 1, into L2 ahead of the dependent levels
   // (K and V, two 128-byte lines each)
   for (int l = 2; l <= t_new; ++l) {
@@ -383,89 +419,99 @@ __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendA
       prefetch_l2(((e & 2) ? a.v_node : a.k_node) + base + (c0 + (e >> 2)) * kD + (e & 1) * (kD / 2));
   }
 
-  float wr[kHalfK];  // W[d][64 * is_v + i]
-  bool w_ready = false;
-  const int kbase = is_v ? kHalfK : 0;
-  for (int l = 1; l <= t_new; ++l) {
+  for (int l = 1; l <= t_new && ok; ++l) {
     const int64_t span_prev = a.span[l - 1];
     const int64_t n_prev = lv_np[l], j0 = lv_j0[l], j1 = lv_j1[l];
     const uint16_t *src = l == 1 ? (is_v ? a.v_tok : a.k_tok) + tok_base
                                  : (is_v ? a.v_node : a.k_node) + (a.row_off[l - 1] + bhi * a.slots[l - 1]) * kD;
     uint16_t *dk = a.k_node + (a.row_off[l] + bhi * a.slots[l]) * kD;
     uint16_t *dv = a.v_node + (a.row_off[l] + bhi * a.slots[l]) * kD;
-    for (int64_t j = j0; j < j1; ++j) {
-      const int64_t c0 = j * a.b, c1 = min(c0 + (int64_t)a.b, n_prev);
-      // the level below's row of child c (tokens through the page table when paged)
-      auto child = [&](int64_t c) -> int64_t { return l == 1 ? tok_row(c) : c; };
-      float sum = 0.f;
+    for (int64_t g0 = j0; g0 < j1 && ok; g0 += umma::kM) {  // up to 128 nodes a product
+      const int64_t g1 = min(j1, g0 + (int64_t)umma::kM);
+      for (int64_t j = g0; j < g1; ++j) {
+        const int64_t c0 = j * a.b, c1 = min(c0 + (int64_t)a.b, n_prev);
+        // the level below's row of child c (tokens through the page table when paged)
+        auto child = [&](int64_t c) -> int64_t { return l == 1 ? tok_row(c) : c; };
+        float sum = 0.f;
 #pragma unroll 16
-      for (int64_t c = c0; c < c1; ++c) {
-        const int64_t r = child(c);
-        if (r >= 0) sum += bf16_lo(src[r * kD + d]);
-      }
-      const float nch = (float)(c1 - c0);
-      if (is_v) {  // token-weighted: the level's last child gets its share tokens / span_prev
-        float wsum = nch;
-        if (c1 == n_prev && c1 > c0) {
-          const int64_t last_tokens = length - (c1 - 1) * span_prev;
-          if (last_tokens < span_prev) {
-            const float f1 = (float)last_tokens / (float)span_prev - 1.f;
-            const int64_t r = child(c1 - 1);
-            sum = __fmaf_rn(f1, r >= 0 ? bf16_lo(src[r * kD + d]) : 0.f, sum);
-            wsum += f1;
+        for (int64_t c = c0; c < c1; ++c) {
+          const int64_t r = child(c);
+          if (r >= 0) sum += bf16_lo(src[r * kD + d]);
+        }
+        const float nch = (float)(c1 - c0);
+        if (is_v) {  // token-weighted: the level's last child gets its share tokens / span_prev
+          float wsum = nch;
+          if (c1 == n_prev && c1 > c0) {
+            const int64_t last_tokens = length - (c1 - 1) * span_prev;
+            if (last_tokens < span_prev) {
+              const float f1 = (float)last_tokens / (float)span_prev - 1.f;
+              const int64_t r = child(c1 - 1);
+              sum = __fmaf_rn(f1, r >= 0 ? bf16_lo(src[r * kD + d]) : 0.f, sum);
+              wsum += f1;
+            }
           }
+          dv[j * kD + d] = (uint16_t)f32_to_bf16_bits(sum / wsum);
+        } else {  // the key mean's three bf16 parts into row j - g0 of A
+          uint32_t p0, p1, p2;
+          umma::split3(sum / nch, p0, p1, p2);
+          const int off = umma::operand_offset((int)(j - g0), d);
+          *reinterpret_cast<uint16_t *>(A + off) = (uint16_t)p0;
+          *reinterpret_cast<uint16_t *>(A + umma::kPartBytes + off) = (uint16_t)p1;
+          *reinterpret_cast<uint16_t *>(A + 2 * umma::kPartBytes + off) = (uint16_t)p2;
         }
-        dv[j * kD + d] = (uint16_t)f32_to_bf16_bits(sum / wsum);
-      } else {
-        mean[d] = sum / nch;
       }
-      if (!w_ready) {  // first node: W^T through shared memory into each thread's registers
-#pragma unroll
-        for (int i = 0; i < kPieces; ++i) {
-          const int e = tid + i * kExtendThreads;
-          const int o = e >> 5, q = e & 31;  // W[o][4q .. 4q+3]
-          Wt[(4 * q + 0) * kD + (o ^ q)] = w[i].x;
-          Wt[(4 * q + 1) * kD + (o ^ q)] = w[i].y;
-          Wt[(4 * q + 2) * kD + (o ^ q)] = w[i].z;
-          Wt[(4 * q + 3) * kD + (o ^ q)] = w[i].w;
-        }
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < kHalfK; ++i) {
-          const int k = kbase + i;
-          wr[i] = Wt[k * kD + (d ^ ((k >> 2) & 31))];
-        }
-        w_ready = true;
+      umma::fence_async_smem();
+      umma::fence_before_sync();
+      __syncthreads();  // the key means in place
+      if (tid == 0) {
+        umma::fence_after_sync();
+        umma::issue_pooler(tmem, smem_u32(A), smem_u32(Bop));
+        umma::commit(bar);
       }
-      __syncthreads();  // the key mean in place
-      const float4 *m4 = reinterpret_cast<const float4 *>(mean + kbase);
-      float acc = 0.f;
-      if (!is_v) {
+      const bool done = __all_sync(0xffffffffu, mbar_wait(bar, ph));  // one answer a warp
+      ph ^= 1u;
+      umma::fence_after_sync();
+      if (done) {  // keys of nodes g0 .. g1-1: warp w reads lanes 32 (w % 4) .., columns 64 (w / 4) ..
+        const int rq = warp & 3, ch = warp >> 2, row = 32 * rq + lane;
+        uint32_t v0[32], v1[32];
+        const uint32_t t0 = tmem + ((uint32_t)(32 * rq) << 16) + 64u * ch;
+        umma::tmem_ld32(t0, v0);
+        umma::tmem_ld32(t0 + 32, v1);
+        umma::tmem_wait_ld();
+        if (row < g1 - g0) {
+          uint4 *dst = reinterpret_cast<uint4 *>(dk + (g0 + row) * kD + 64 * ch);
 #pragma unroll
-        for (int i = 0; i < kHalfK / 4; ++i) {
-          const float4 m = m4[i];
-          acc = __fmaf_rn(m.x, wr[4 * i + 0], acc);
-          acc = __fmaf_rn(m.y, wr[4 * i + 1], acc);
-          acc = __fmaf_rn(m.z, wr[4 * i + 2], acc);
-          acc = __fmaf_rn(m.w, wr[4 * i + 3], acc);
-        }
-        part[d] = acc;
-      }
-      __syncthreads();  // the first half of every key output in place
-      if (is_v) {
-        acc = part[d];
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(pack_bf16x2(__uint_as_float(v0[8 * q]), __uint_as_float(v0[8 * q + 1])),
+                                pack_bf16x2(__uint_as_float(v0[8 * q + 2]), __uint_as_float(v0[8 * q + 3])),
+                                pack_bf16x2(__uint_as_float(v0[8 * q + 4]), __uint_as_float(v0[8 * q + 5])),
+                                pack_bf16x2(__uint_as_float(v0[8 * q + 6]), __uint_as_float(v0[8 * q + 7])));
 #pragma unroll
-        for (int i = 0; i < kHalfK / 4; ++i) {
-          const float4 m = m4[i];
-          acc = __fmaf_rn(m.x, wr[4 * i + 0], acc);
-          acc = __fmaf_rn(m.y, wr[4 * i + 1], acc);
-          acc = __fmaf_rn(m.z, wr[4 * i + 2], acc);
-          acc = __fmaf_rn(m.w, wr[4 * i + 3], acc);
+          for (int q = 0; q < 4; ++q)
+            dst[4 + q] = make_uint4(pack_bf16x2(__uint_as_float(v1[8 * q]), __uint_as_float(v1[8 * q + 1])),
+                                    pack_bf16x2(__uint_as_float(v1[8 * q + 2]), __uint_as_float(v1[8 * q + 3])),
+                                    pack_bf16x2(__uint_as_float(v1[8 * q + 4]), __uint_as_float(v1[8 * q + 5])),
+                                    pack_bf16x2(__uint_as_float(v1[8 * q + 6]), __uint_as_float(v1[8 * q + 7])));
         }
-        dk[j * kD + d] = (uint16_t)f32_to_bf16_bits(acc);
       }
-      __syncthreads();  // mean and part are rewritten next, and the next level reads these rows
+      if (!__syncthreads_and(done)) {
+        // the product did not complete within the wait limit: report it; the walk stops
+        if (tid == 0) {
+          if (a.err) atomicOr(a.err, kErrTimeout);
+          atomicOr(&g_build_err, kErrTimeout);
+          mbar_wait(bar, ph ^ 1u);  // a last bounded wait before the accumulator is freed
+        }
+        ok = false;
+      }
+      umma::fence_before_sync();
+      __syncthreads();  // A is rewritten next, and the next level reads these rows
     }
+  }
+  umma::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    umma::fence_after_sync();
+    umma::tmem_dealloc(tmem, umma::kTmemCols);
   }
 }
 
@@ -535,17 +581,11 @@ int configure_smem() {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return (int)e;
   if (configured_device == dev) return 0;
-  e = cudaFuncSetAttribute(build_level_kernel<kNodesPerWarp, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)build_smem(kNodesPerWarp));
+  e = cudaFuncSetAttribute(build_level_mma_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kMmaSmem);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(build_level_kernel<kFewNodes, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)build_smem(kFewNodes));
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(build_level_kernel<kNodesPerWarp, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)build_smem(kNodesPerWarp));
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(build_level_kernel<kFewNodes, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)build_smem(kFewNodes));
+    e = cudaFuncSetAttribute(build_level_mma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kMmaSmem);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(extend_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kExtendSmem);
   if (e == cudaSuccess)
@@ -556,6 +596,14 @@ int configure_smem() {
 }
 
 }  // namespace
+
+int read_build_errors(uint32_t *bits) {
+  uint32_t v = 0u, zero = 0u;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_build_err, sizeof(v));
+  if (e == cudaSuccess && v != 0u) e = cudaMemcpyToSymbol(g_build_err, &zero, sizeof(zero));
+  *bits = v;
+  return (int)e;
+}
 
 int launch_rope_table(void *ws, int rows, double base, void *stream) {
   auto *hdr = reinterpret_cast<WsHeader *>(ws);
@@ -597,17 +645,12 @@ int launch_build_level(const TreeGeom &g, const recsa_tree &t, int level, int64_
   a.pooler = t.pooler;
   const int rc = configure_smem();
   if (rc != 0) return rc;
-  const int64_t nodes = (int64_t)a.bh * a.nj;
-  const int64_t full_grid = (int64_t)sm_count() * 2;
-  // one pass of warps with a node each when it fits, else 8 nodes a warp over a grid of 2 CTAs
-  // per SM; the paged instances read level 1 through the page table
-  const bool few = nodes <= full_grid * kBuildWarps * kFewNodes;
-  const int npw = few ? kFewNodes : kNodesPerWarp;
-  const int64_t grid = few ? ceil_div(nodes, kBuildWarps * kFewNodes)
-                           : std::min<int64_t>(ceil_div(nodes, kBuildWarps * kNodesPerWarp), full_grid);
-  auto kern = few ? (a.pages ? build_level_kernel<kFewNodes, true> : build_level_kernel<kFewNodes, false>)
-                  : (a.pages ? build_level_kernel<kNodesPerWarp, true> : build_level_kernel<kNodesPerWarp, false>);
-  kern<<<(unsigned)grid, kBuildThreads, build_smem(npw), (cudaStream_t)stream>>>(a);
+  // tiles of 128 nodes over a persistent grid of one CTA per SM; the paged instance reads
+  // level 1 through the page table
+  const int64_t tiles = ceil_div((int64_t)a.bh * a.nj, (int64_t)umma::kM);
+  const int64_t grid = std::min<int64_t>(tiles, (int64_t)sm_count());
+  auto kern = a.pages ? build_level_mma_kernel<true> : build_level_mma_kernel<false>;
+  kern<<<(unsigned)grid, kMmaThreads, kMmaSmem, (cudaStream_t)stream>>>(a);
   return (int)cudaGetLastError();
 }
 

@@ -51,6 +51,9 @@ int levels_for(int64_t length, int b);  // T(length)
 
 // Launchers (return cudaError_t as int; 0 = success)
 int launch_rope_table(void *ws, int rows, double base, void *stream);
+// Read and clear the build kernels' device error word (kErrTimeout when a wait on the tensor
+// cores gave up); returns a cudaError_t.
+int read_build_errors(uint32_t *bits);
 int launch_build_level(const TreeGeom &g, const recsa_tree &t, int level, int64_t length, int64_t j0, int64_t j1,
                        void *stream);
 int launch_append(const TreeGeom &g, const recsa_tree &t, const void *k_new, const void *v_new, int64_t at,

@@ -59,6 +59,7 @@ struct TBarrier {
 };
 
 extern thread_local int t_tid, t_block, t_crank, t_cs, t_grid;
+extern int g_nt;  // threads per CTA
 extern thread_local long t_cluster_gen;  // cluster-barrier generation this thread arrived at
 extern thread_local unsigned char *t_smem;
 extern std::vector<unsigned char *> g_cluster_smem;  // per cluster rank
@@ -72,8 +73,8 @@ extern std::vector<Where> g_where;            // per (rank, tid)
 void report_and_abort(const char *why);
 
 inline void TBarrier::wait(int line) {
-  g_where[t_crank * 256 + t_tid].line = line;
-  g_where[t_crank * 256 + t_tid].what = name.c_str();
+  g_where[t_crank * g_nt + t_tid].line = line;
+  g_where[t_crank * g_nt + t_tid].what = name.c_str();
   std::unique_lock<std::mutex> lk(mu);
   const long my = gen;
   if (++arrived == count) {
@@ -92,8 +93,8 @@ inline void TBarrier::wait(int line) {
 }
 
 inline long TBarrier::arrive(int line) {
-  g_where[t_crank * 256 + t_tid].line = line;
-  g_where[t_crank * 256 + t_tid].what = "cluster-arrive";
+  g_where[t_crank * g_nt + t_tid].line = line;
+  g_where[t_crank * g_nt + t_tid].what = "cluster-arrive";
   std::lock_guard<std::mutex> lk(mu);
   const long my = gen;
   if (++arrived == count) {
@@ -105,8 +106,8 @@ inline long TBarrier::arrive(int line) {
 }
 
 inline void TBarrier::wait_gen(long my, int line) {
-  g_where[t_crank * 256 + t_tid].line = line;
-  g_where[t_crank * 256 + t_tid].what = name.c_str();
+  g_where[t_crank * g_nt + t_tid].line = line;
+  g_where[t_crank * g_nt + t_tid].what = name.c_str();
   std::unique_lock<std::mutex> lk(mu);
   if (!cv.wait_for(lk, std::chrono::seconds(20), [&] { return gen != my; })) {
     lk.unlock();
@@ -124,13 +125,13 @@ struct ThreadIdx { unsigned x; };
 #define gridDim (ThreadIdx{(unsigned)emu::t_grid})
 
 #define __syncthreads() emu::g_cta_bar[emu::t_crank].wait(__LINE__)
-#define __syncwarp(...) emu::g_warp_bar[emu::t_crank * 8 + emu::t_tid / 32].wait(__LINE__)
+#define __syncwarp(...) emu::g_warp_bar[emu::t_crank * (emu::g_nt / 32) + emu::t_tid / 32].wait(__LINE__)
 
 namespace emu {
 template <typename T>
 inline T warp_exchange(T v, int src, int line) {
   static_assert(sizeof(T) == 4, "32-bit values only");
-  const int w = t_crank * 8 + t_tid / 32, lane = t_tid & 31;
+  const int w = t_crank * (g_nt / 32) + t_tid / 32, lane = t_tid & 31;
   uint32_t u;
   std::memcpy(&u, &v, 4);
   g_warp_slot[w * 32 + lane] = u;
@@ -146,7 +147,7 @@ inline T warp_exchange(T v, int src, int line) {
 #define __shfl_xor_sync(m, v, x) emu::warp_exchange((v), (emu::t_tid & 31) ^ (x), __LINE__)
 namespace emu {
 inline unsigned ballot(bool p, int line) {
-  const int w = t_crank * 8 + t_tid / 32, lane = t_tid & 31;
+  const int w = t_crank * (g_nt / 32) + t_tid / 32, lane = t_tid & 31;
   g_warp_slot[w * 32 + lane] = p ? 1u : 0u;
   g_warp_bar[w].wait(line);
   unsigned b = 0;
@@ -156,6 +157,7 @@ inline unsigned ballot(bool p, int line) {
 }
 }  // namespace emu
 #define __ballot_sync(m, p) emu::ballot((p), __LINE__)
+#define __all_sync(m, p) (emu::ballot((p), __LINE__) == 0xffffffffu)
 
 inline int __popc(uint32_t x) { return __builtin_popcount(x); }
 inline int __clz(uint32_t x) { return x ? __builtin_clz(x) : 32; }
@@ -194,7 +196,7 @@ inline long min(long a, long b) { return a < b ? a : b; }
 inline long max(long a, long b) { return a > b ? a : b; }
 namespace emu {
 inline unsigned warp_reduce(unsigned v, bool is_max, int line) {
-  const int w = t_crank * 8 + t_tid / 32, lane = t_tid & 31;
+  const int w = t_crank * (g_nt / 32) + t_tid / 32, lane = t_tid & 31;
   g_warp_slot[w * 32 + lane] = v;
   g_warp_bar[w].wait(line);
   unsigned r = g_warp_slot[w * 32];
@@ -208,5 +210,33 @@ inline unsigned warp_reduce(unsigned v, bool is_max, int line) {
 }  // namespace emu
 #define __reduce_max_sync(m, v) emu::warp_reduce((v), true, __LINE__)
 #define __reduce_min_sync(m, v) emu::warp_reduce((v), false, __LINE__)
+namespace emu {
+// __syncthreads_and: every thread's predicate, one barrier, the AND to all
+extern std::vector<uint32_t> g_cta_pred;  // per (rank, tid)
+inline int cta_and(bool p, int line) {
+  g_cta_pred[t_crank * g_nt + t_tid] = p ? 1u : 0u;
+  g_cta_bar[t_crank].wait(line);
+  int all = 1;
+  for (int i = 0; i < g_nt; ++i) all &= (int)g_cta_pred[t_crank * g_nt + i];
+  g_cta_bar[t_crank].wait(line);
+  return all;
+}
+// mbarrier with transaction counts: a phase completes when its arrivals and its expected
+// bytes are all in
+struct MBar {
+  std::mutex mu;
+  int count = 0, pending = 0;
+  long tx = 0;
+  long completed = 0;  // phases completed so far
+};
+MBar &mbar_of(const void *p);
+inline void mbar_complete_if_done(MBar &b) {
+  if (b.pending == 0 && b.tx == 0) {
+    ++b.completed;
+    b.pending = b.count;
+  }
+}
+}  // namespace emu
+#define __syncthreads_and(p) emu::cta_and((p), __LINE__)
 inline unsigned max(unsigned a, unsigned b) { return a > b ? a : b; }
 inline unsigned min(unsigned a, unsigned b) { return a < b ? a : b; }

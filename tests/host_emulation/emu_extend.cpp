@@ -1,8 +1,8 @@
 // Runs the append kernel (extend_kernel: one CTA of 256 threads per (sequence, KV head)) or, with
-// "mode 1", every level of the tree build (build_level_kernel, one launch per level, a grid of
-// "grid" CTAs striding over the level's nodes, "npw" nodes a warp) on host threads, one
+// "mode 1", every level of the tree build (build_level_mma_kernel, one launch per level, a grid of
+// at most "grid" CTAs of 512 threads striding over tiles of 128 nodes) on host threads, one
 // std::thread per CUDA thread, over inputs read from a case directory, and writes the caches and
-// the node arena back there.  Test infrastructure: it checks the kernels' barriers (every thread
+// the node arena back there.  The tensor-core steps run through host versions (emu_umma_ops.h).  Test infrastructure: it checks the kernels' barriers (every thread
 // reaches each one), their memory accesses (AddressSanitizer) and their results, without a GPU.
 //
 // usage: emu_extend <case dir>
@@ -10,7 +10,10 @@
 //                     ints); optional "seq_len" (one per sequence) and "pages" (the page table)
 //   <dir>/{k_tok,v_tok,k_node,v_node,k_new,v_new}.bin bf16 arrays, <dir>/pooler.bin fp32 [128][128]
 //   writes <dir>/{k_tok,v_tok,k_node,v_node}_out.bin
+#include <cmath>
 #include <fstream>
+#include <memory>
+#include <mutex>
 #include <map>
 #include <sstream>
 #include <thread>
@@ -19,6 +22,17 @@
 
 namespace emu {
 thread_local int t_tid, t_block, t_crank, t_cs, t_grid = 1;
+int g_nt = 256;
+thread_local float *t_tmem;
+std::vector<uint32_t> g_cta_pred;
+std::mutex g_mbar_mu;
+std::map<const void *, std::unique_ptr<MBar>> g_mbars;
+MBar &mbar_of(const void *p) {
+  std::lock_guard<std::mutex> lk(g_mbar_mu);
+  auto &slot = g_mbars[p];
+  if (!slot) slot.reset(new MBar());
+  return *slot;
+}
 thread_local long t_cluster_gen = -1;
 thread_local unsigned char *t_smem;
 std::vector<unsigned char *> g_cluster_smem;
@@ -34,7 +48,7 @@ void report_and_abort(const char *why) {
   static std::mutex m;
   std::lock_guard<std::mutex> lk(m);
   fprintf(stderr, "STALL: %s\n", why);
-  for (int t = 0; t < 256; ++t)
+  for (int t = 0; t < g_nt; ++t)
     fprintf(stderr, "  thread %d waits at %s:%d\n", t, (const char *)g_where[t].what, (int)g_where[t].line);
   fflush(stderr);
   _exit(3);
@@ -64,19 +78,26 @@ void write_bin(const std::string &path, const std::vector<T> &v) {
 }
 
 template <typename Kernel>
-void run_block(Kernel kernel, size_t smem_bytes, int block, int grid) {
+void run_block(Kernel kernel, size_t smem_bytes, int block, int grid, int nthreads) {
   using namespace emu;
   std::vector<unsigned char> smem(smem_bytes, 0xAB);
+  std::vector<float> tmem(128 * 512, std::nanf(""));
+  g_nt = nthreads;
+  {
+    std::lock_guard<std::mutex> lk(g_mbar_mu);
+    g_mbars.clear();
+  }
   g_smem_bytes = smem.size();
   g_cluster_smem.assign(1, smem.data());
   g_cta_bar = std::vector<TBarrier>(1);
-  g_cta_bar[0].init(256, "syncthreads");
-  g_warp_bar = std::vector<TBarrier>(8);
+  g_cta_bar[0].init(nthreads, "syncthreads");
+  g_cta_pred.assign(nthreads, 0u);
+  g_warp_bar = std::vector<TBarrier>(nthreads / 32);
   for (auto &w : g_warp_bar) w.init(32, "warp");
-  g_warp_slot.assign(8 * 32, 0);
-  g_where = std::vector<Where>(256);
+  g_warp_slot.assign(nthreads, 0);
+  g_where = std::vector<Where>(nthreads);
   std::vector<std::thread> th;
-  for (int t = 0; t < 256; ++t)
+  for (int t = 0; t < nthreads; ++t)
     th.emplace_back([&, t] {
       t_tid = t;
       t_crank = 0;
@@ -84,6 +105,7 @@ void run_block(Kernel kernel, size_t smem_bytes, int block, int grid) {
       t_block = block;
       t_grid = grid;
       t_smem = smem.data();
+      t_tmem = tmem.data();
       kernel();
       g_where[t].line = -1;
       g_where[t].what = "exited";
@@ -150,7 +172,7 @@ int main(int argc, char **argv) {
   const int blocks = (int)kv["batch"] * a.hkv;
   if ((int)kv["mode"] == 1) {  // the whole build, level by level, over `length` tokens
     const int64_t length = (int64_t)kv["length"];
-    const int npw = (int)kv["npw"], grid_cap = (int)kv["grid"];
+    const int grid_cap = (int)kv["grid"];
     for (int l = 1; l <= a.levels; ++l) {
       BuildArgs g = {};
       const bool from_tokens = l == 1;
@@ -177,25 +199,21 @@ int main(int argc, char **argv) {
       g.pages_per_seq = paged ? a.capacity >> a.page_shift : 0;
       g.num_pages = a.num_pages;
       g.pooler = pooler.data();
-      const int64_t per_block = (int64_t)kBuildWarps * npw;
-      const int grid = (int)std::min<int64_t>((g.bh * g.nj + per_block - 1) / per_block, grid_cap);
+      const int64_t tiles = (g.bh * g.nj + umma::kM - 1) / umma::kM;
+      const int grid = (int)std::min<int64_t>(tiles, grid_cap);
       for (int blk = 0; blk < grid; ++blk) {
-        if (npw == 1 && g.pages)
-          run_block([&] { build_level_kernel<kFewNodes, true>(g); }, build_smem(kFewNodes), blk, grid);
-        else if (npw == 1)
-          run_block([&] { build_level_kernel<kFewNodes, false>(g); }, build_smem(kFewNodes), blk, grid);
-        else if (g.pages)
-          run_block([&] { build_level_kernel<kNodesPerWarp, true>(g); }, build_smem(kNodesPerWarp), blk, grid);
+        if (g.pages)
+          run_block([&] { build_level_mma_kernel<true>(g); }, kMmaSmem, blk, grid, kMmaThreads);
         else
-          run_block([&] { build_level_kernel<kNodesPerWarp, false>(g); }, build_smem(kNodesPerWarp), blk, grid);
+          run_block([&] { build_level_mma_kernel<false>(g); }, kMmaSmem, blk, grid, kMmaThreads);
       }
     }
   } else {
     for (int blk = 0; blk < blocks; ++blk) {
       if (paged)
-        run_block([&] { extend_kernel<true>(a); }, kExtendSmem, blk, blocks);
+        run_block([&] { extend_kernel<true>(a); }, kExtendSmem, blk, blocks, kExtendThreads);
       else
-        run_block([&] { extend_kernel<false>(a); }, kExtendSmem, blk, blocks);
+        run_block([&] { extend_kernel<false>(a); }, kExtendSmem, blk, blocks, kExtendThreads);
     }
   }
   write_bin(dir + "/k_tok_out.bin", ktok);

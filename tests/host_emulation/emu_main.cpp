@@ -18,6 +18,8 @@
 
 namespace emu {
 thread_local int t_tid, t_block, t_crank, t_cs, t_grid = 1;
+int g_nt = 256;
+std::vector<uint32_t> g_cta_pred;
 thread_local long t_cluster_gen = -1;
 thread_local unsigned char *t_smem;
 std::vector<unsigned char *> g_cluster_smem;

@@ -170,9 +170,9 @@ def test_append_into_a_paged_cache(emu_bin, tmp_path, P):
     _run(emu_bin, tmp_path, [600, 301], 1, 5, 4, P=P, per_seq=True, seed=P)
 
 
-def _run_build(emu_bin, tmp_path, lens, hkv, b, npw, grid, P=None, per_seq=False, seed=3):
-    """The level-build kernel over every level (grid-stride over `grid` CTAs, `npw` nodes a
-    warp) on the CPU; each sequence's node rows against the oracle's tree over its tokens."""
+def _run_build(emu_bin, tmp_path, lens, hkv, b, grid, P=None, per_seq=False, seed=3):
+    """The level-build kernel over every level (at most `grid` CTAs striding over the tiles of
+    128 nodes) on the CPU; each sequence's node rows against the oracle's tree over its tokens."""
     B, L = len(lens), max(lens)
     cap = -(-L // P) * P if P else L
     inp = I.random_case(B, L, hkv, hkv * 4, 0, seed=seed, capacity=cap)
@@ -181,7 +181,7 @@ def _run_build(emu_bin, tmp_path, lens, hkv, b, npw, grid, P=None, per_seq=False
     p = R.params(num_kv_heads=hkv, num_q_heads=hkv * 4, branching=b, top_k=2)
     node_rows, levels_cap, offs = R.tree_layout(p, B, cap)
     slots = [cap] + [math.ceil(cap / b ** lv) for lv in range(1, levels_cap + 1)]
-    prm = dict(mode=1, length=L, npw=npw, grid=grid, batch=B, hkv=hkv, b=b, capacity=cap, at=0, chunk=0,
+    prm = dict(mode=1, length=L, grid=grid, batch=B, hkv=hkv, b=b, capacity=cap, at=0, chunk=0,
                levels=len(O.level_counts(L, b)) - 1, page_shift=0, num_pages=0)
     k_in, v_in, pages = kb, vb, None
     if P:
@@ -196,7 +196,7 @@ def _run_build(emu_bin, tmp_path, lens, hkv, b, npw, grid, P=None, per_seq=False
             for j in range(pps):
                 k_in[pages[s, j]] = kb[s, :, j * P:(j + 1) * P]
                 v_in[pages[s, j]] = vb[s, :, j * P:(j + 1) * P]
-    d = tmp_path / f"build_{B}_{hkv}_{L}_{b}_{npw}_{grid}_{P}_{int(per_seq)}"
+    d = tmp_path / f"build_{B}_{hkv}_{L}_{b}_{grid}_{P}_{int(per_seq)}"
     d.mkdir()
     span = [min(b ** lv, 1 << 62) for lv in range(R.MAX_LEVELS + 1)]
     with open(d / "params.txt", "w") as f:
@@ -234,10 +234,10 @@ def _run_build(emu_bin, tmp_path, lens, hkv, b, npw, grid, P=None, per_seq=False
     assert total > 0 and mism <= total * 1e-2
 
 
-@pytest.mark.parametrize("npw,grid", [(8, 2), (1, 1000)])  # a grid that strides, and a node per warp
-def test_level_build_matches_oracle(emu_bin, tmp_path, npw, grid):
-    _run_build(emu_bin, tmp_path, [1000, 1000], 2, 4, npw, grid)
+@pytest.mark.parametrize("grid", [1, 1000])  # one CTA striding over every tile, and a CTA a tile
+def test_level_build_matches_oracle(emu_bin, tmp_path, grid):
+    _run_build(emu_bin, tmp_path, [1000, 1000], 2, 4, grid)
 
 
 def test_level_build_with_per_sequence_lengths_and_pages(emu_bin, tmp_path):
-    _run_build(emu_bin, tmp_path, [700, 0, 301, 64], 1, 4, 8, 3, P=8, per_seq=True)
+    _run_build(emu_bin, tmp_path, [700, 0, 301, 64], 1, 4, 3, P=8, per_seq=True)
