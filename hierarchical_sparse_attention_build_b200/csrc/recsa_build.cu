@@ -67,6 +67,11 @@ struct PagedRows {
   }
 };
 
+// A run of rows into L2 (16-byte aligned start, a multiple of 16 bytes).
+__device__ __forceinline__ void prefetch_rows_l2(const void *p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // One child row piece (the lane's 4 dims): through the read-only path for a level written by
 // an earlier launch, an ordinary load for one this kernel may have written.
 template <bool kReadOnly>
@@ -217,6 +222,22 @@ __global__ void __launch_bounds__(kMmaThreads, 1) build_level_mma_kernel(const B
       const int row = warp * kMmaNodesPerWarp + n;
       int64_t bhi, j, length, n_prev;
       float ks[4] = {0.f, 0.f, 0.f, 0.f}, vs[4] = {0.f, 0.f, 0.f, 0.f};
+      // the warp's next node's children (two contiguous runs, K and V) into L2 while this
+      // node's stream: the loads of the next node then wait on L2, not DRAM (a paged token
+      // cache scatters them, so it is not prefetched)
+      if (!kPaged && lane == 0) {
+        int64_t bh2, j2, len2, np2;
+        const int64_t nid = n + 1 < kMmaNodesPerWarp ? tile * umma::kM + row + 1
+                                                     : (tile + gridDim.x) * umma::kM + warp * kMmaNodesPerWarp;
+        if (locate(nid, bh2, j2, len2, np2)) {
+          const int64_t c0 = j2 * a.b, cnt = min(c0 + (int64_t)a.b, np2) - c0;
+          if (cnt > 0) {
+            const int64_t r0 = (a.src_row_off + bh2 * a.src_slots + c0) * kD;
+            prefetch_rows_l2(a.src_k + r0, (uint32_t)(cnt * kD * 2));
+            prefetch_rows_l2(a.src_v + r0, (uint32_t)(cnt * kD * 2));
+          }
+        }
+      }
       if (locate(tile * umma::kM + row, bhi, j, length, n_prev)) {
         const int64_t c0 = j * a.b;
         const int64_t c1 = min(c0 + (int64_t)a.b, n_prev);

@@ -83,7 +83,9 @@ def extract_extend(src_path: str, out_path: str) -> None:
                  os.path.join(os.path.dirname(out_path), "umma_extracted.h"))
     for old, new in (("#include <cuda_runtime.h>", ""), ('#include "recsa_device.cuh"', '#include "emu_device.h"'),
                      ('#include "recsa_umma.cuh"', '#include "umma_extracted.h"'),
-                     ('asm volatile("prefetch.global.L2 [%0];" ::"l"(p));', "(void)p;")):
+                     ('asm volatile("prefetch.global.L2 [%0];" ::"l"(p));', "(void)p;"),
+                     ('asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");',
+                      "(void)p;\n  (void)bytes;")):
         if old not in text:
             raise ValueError(f"expected text not found in the build source: {old}")
         text = text.replace(old, new)
