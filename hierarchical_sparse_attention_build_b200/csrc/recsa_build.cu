@@ -322,10 +322,19 @@ __global__ void __launch_bounds__(kMmaThreads, 1) build_level_mma_kernel(const B
 // them are those nodes' ancestors).  A thread owns one dimension of the key (threads
 // 0..127) or of the value (128..255): it sums that dimension over the node's children and
 // forms its mean, in the level build's operation order.  The level's key means (up to 128
-// nodes at a time) go to the A operand and one thread issues the same split-bf16 pooler
-// product as the level build, so the extended tree equals a full build bit for bit.  Rows
+// nodes at a time) go to an operand and a thread of a warp of its own issues the level
+// build's split-bf16 pooler product with the operands' roles exchanged (W as A, the means as
+// B, N = the node count rounded up to 16), so the extended tree equals a full build bit for
+// bit.  Rows
 // written at level l are read at level l+1 by other threads of the same CTA after a
 // __syncthreads; no two CTAs touch the same rows.
+//
+// The walk's critical path is one product a level (48 MMA instructions, ~2.5K cycles).  What
+// else is on it is kept short on the path of a single token (one node a level): the node's
+// children other than the last are unchanged rows, summed ahead (the next level's while this
+// level's product runs), and its last child is the node rebuilt one level below, which the
+// thread owning the dimension already holds (key thread d reads accumulator lane d, value
+// thread d formed the value); the sum then continues with it in the children's order.
 struct ExtendArgs {
   const uint4 *k_new, *v_new;   // [B][C][Hkv][128] bf16, as 16-byte pieces
   uint16_t *k_tok, *v_tok;      // [B][Hkv][capacity][128]
@@ -342,9 +351,15 @@ struct ExtendArgs {
   int64_t slots[kMaxLevels + 1];
   int64_t span[kMaxLevels + 1];
 };
-constexpr int kExtendThreads = 2 * kD;  // one thread per key dimension and per value dimension
-// the A and B operands of the pooler product, the product's barrier and the TMEM address, and
-// per level the rebuilt node range [j0, j1) and the node count of the level below
+// One thread per key dimension and per value dimension, and one more warp that allocates the
+// accumulator and issues the pooler product: a thread issuing the product's 48 MMA
+// instructions is held for about as long as the product runs (~2.5K cycles, measured), so the
+// dimension threads work out the next level's head start meanwhile.
+constexpr int kExtendDimThreads = 2 * kD;
+constexpr int kExtendThreads = kExtendDimThreads + 32;
+constexpr int kExtendIssuer = kExtendDimThreads;  // the issuing thread (lane 0 of the last warp)
+// W's and the means' operands of the pooler product, the product's barrier and the TMEM
+// address, and per level the rebuilt node range [j0, j1) and the node count of the level below
 constexpr size_t kExtendSmem = 2 * (size_t)umma::kOperandBytes + 128 + 3 * (kMaxLevels + 1) * sizeof(int64_t);
 
 // x / y and ceil(x / y) for x >= 0, y >= 1, in 32 bits whenever the operands fit (a 64-bit
@@ -363,7 +378,7 @@ __device__ __forceinline__ void prefetch_l2(const void *p) {
 template <bool kPaged>
 __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendArgs a) {
   extern __shared__ __align__(128) unsigned char smem_u8[];
-  unsigned char *A = smem_u8, *Bop = smem_u8 + umma::kOperandBytes;
+  unsigned char *Wop = smem_u8, *Mop = smem_u8 + umma::kOperandBytes;  // W's parts, the key means' parts
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem_u8 + 2 * umma::kOperandBytes);
   uint32_t *tmem_s = reinterpret_cast<uint32_t *>(bar + 1);
   int64_t *lv_j0 = reinterpret_cast<int64_t *>(smem_u8 + 2 * umma::kOperandBytes + 128);  // per level: nodes
@@ -389,32 +404,108 @@ __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendA
   // level l rebuilds nodes [j0, j1): those whose spans meet the new tokens (a level that
   // becomes new is built whole); the first warp works the levels out side by side, once,
   // rather than every thread on the walk's dependent path
-  if (tid < 32)
+  const int warp = tid >> 5;
+  const bool dims = tid < kExtendDimThreads;  // a dimension thread (else the issuing warp)
+  if (warp == 0)
     for (int l = tid + 1; l <= t_new; l += 32) {
       lv_j0[l] = l <= t_old ? div_nn(at, a.span[l]) : 0;
       lv_j1[l] = ceil_div_nn(length, a.span[l]);
       lv_np[l] = ceil_div_nn(length, a.span[l - 1]);
     }
+  if (tid == 32) {
+    mbar_init(bar, 1);
+    mbar_fence_init();
+  }
   // token t of this (sequence, head): row tok_base + tok_row(t), -1 for a page outside the pool
   const int64_t h = bhi % a.hkv;
   const int64_t tok_base = kPaged ? (h << a.page_shift) * kD : bhi * a.capacity * kD;
   const PagedRows paged{kPaged ? a.pages + (bhi / a.hkv) * (a.capacity >> a.page_shift) : nullptr,
                         (int64_t)a.hkv << a.page_shift, a.page_shift, a.num_pages};
   auto tok_row = [&](int64_t t) -> int64_t { return kPaged ? paged(t) : t; };
-
-  const int warp = tid >> 5, lane = tid & 31;
-  if (warp == 0) {
+  // level l's rows of this (sequence, head), the thread's half (K or V); level 0 = the tokens
+  auto level_rows = [&](int l) -> uint16_t * {
+    return l == 0 ? (is_v ? a.v_tok : a.k_tok) + tok_base
+                  : (is_v ? a.v_node : a.k_node) + (a.row_off[l] + bhi * a.slots[l]) * kD;
+  };
+  // The single-token path: a level rebuilds one node whose last child is the one rebuilt
+  // below (at level 1: the one new token).  `carry` is that child's dimension d as stored
+  // (bf16), valid while `have_carry`.
+  float carry = 0.f;
+  bool have_carry = false;
+  if (dims && a.chunk == 1 && t_new >= 1 && tok_row(at) >= 0) {
+    const int64_t s = bhi / a.hkv;
+    const uint16_t *src = reinterpret_cast<const uint16_t *>(is_v ? a.v_new : a.k_new);
+    carry = bf16_lo(__ldg(src + ((s * a.hkv + h) * kD + d)));
+    have_carry = true;
+  }
+  __syncthreads();  // the level ranges are in place
+  // the sum of children [c0, c1) of a node of level l (rows of level l-1, in order), this
+  // thread's dim: 16 rows' loads in flight at a time, then their adds in child order (a loop
+  // with a run-time trip count would leave a partial node's rows to a rolled remainder loop,
+  // one L2 round trip each)
+  auto child_sum = [&](int l, int64_t c0, int64_t c1) -> float {
+    const uint16_t *src = level_rows(l - 1);
+    float sum = 0.f;
+    for (int64_t cb = c0; cb < c1; cb += 16) {
+      float x[16];
+      bool in[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int64_t r = cb + i < c1 ? (l == 1 ? tok_row(cb + i) : cb + i) : -1;
+        in[i] = r >= 0;
+        x[i] = in[i] ? bf16_lo(src[r * kD + d]) : 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (in[i]) sum += x[i];
+    }
+    return sum;
+  };
+  // The single-token path's head start at level l, worked out while the level below is
+  // still in progress: the sum over the node's children before the last, the child count,
+  // and for a value the share of a last child that covers fewer tokens than its span (the
+  // same terms, in the same order, as for a node summed whole below).
+  struct Head {
+    float pre, nch, f1, wsum;
+    bool part;          // the last child gets the share f1 + 1
+    uint16_t *v_dst;    // this thread's element of the node's value row
+  };
+  auto head_start = [&](int l) -> Head {
+    Head hs{0.f, 1.f, 0.f, 1.f, false, nullptr};
+    if (!dims || l > t_new || lv_j1[l] - lv_j0[l] != 1) return hs;
+    const int64_t j = lv_j0[l], n_prev = lv_np[l];
+    const int64_t c0 = j * a.b, c1 = min(c0 + (int64_t)a.b, n_prev);
+    hs.pre = child_sum(l, c0, c1 - 1);
+    hs.nch = (float)(c1 - c0);
+    hs.wsum = hs.nch;
+    const int64_t last_tokens = length - (c1 - 1) * a.span[l - 1];
+    if (last_tokens < a.span[l - 1]) {
+      hs.part = true;
+      hs.f1 = (float)last_tokens / (float)a.span[l - 1] - 1.f;
+      hs.wsum += hs.f1;
+    }
+    hs.v_dst = a.v_node + (a.row_off[l] + bhi * a.slots[l] + j) * kD + d;
+    return hs;
+  };
+  if (!dims) {
+    // the issuing warp, while the others stage W: every child row the walk reads into L2
+    // ahead of the dependent levels (K and V, two 128-byte lines each; level 1 only on the
+    // single-token path, a node's token rows), then the accumulator
+    const int lane = tid & 31;
+    for (int l = 1; l <= t_new; ++l) {
+      const int64_t c0 = lv_j0[l] * a.b, c1 = min(lv_j1[l] * a.b, lv_np[l]);
+      if (l == 1 && (kPaged || !(a.chunk == 1 && lv_j1[1] - lv_j0[1] == 1))) continue;
+      const uint16_t *kb = l == 1 ? a.k_tok + tok_base : a.k_node + (a.row_off[l - 1] + bhi * a.slots[l - 1]) * kD;
+      const uint16_t *vb = l == 1 ? a.v_tok + tok_base : a.v_node + (a.row_off[l - 1] + bhi * a.slots[l - 1]) * kD;
+      for (int64_t e = lane; e < (c1 - c0) * 4; e += 32)
+        prefetch_l2(((e & 2) ? vb : kb) + (c0 + (e >> 2)) * kD + (e & 1) * (kD / 2));
+    }
     umma::tmem_alloc(tmem_s, umma::kTmemCols);
     umma::tmem_relinquish();
-  }
-  if (tid == 32) {
-    mbar_init(bar, 1);
-    mbar_fence_init();
-  }
-  umma::load_pooler_operand<kExtendThreads>(a.pooler, Bop, tid);  // W, the B operand, in its three parts
-  {
+  } else {
+    umma::load_pooler_operand<kExtendDimThreads, 16>(a.pooler, Wop, tid);  // W's three parts
     const int64_t s = bhi / a.hkv;
-    for (int64_t e = tid; e < (int64_t)a.chunk * 16; e += kExtendThreads) {  // 16 pieces a row
+    for (int64_t e = tid; e < (int64_t)a.chunk * 16; e += kExtendDimThreads) {  // 16 pieces a row
       const int64_t src = ((s * a.chunk + (e >> 4)) * a.hkv + h) * 16 + (e & 15);
       const int64_t row = tok_row(at + (e >> 4));
       if (row < 0) continue;
@@ -425,112 +516,121 @@ __global__ void __launch_bounds__(kExtendThreads, 1) extend_kernel(const ExtendA
   }
   umma::fence_async_smem();
   umma::fence_before_sync();
-  __syncthreads();  // the level ranges, W and the TMEM address are in place, and the appended rows are
-                    // read below by other threads
+  __syncthreads();  // W and the TMEM address are in place, and the appended rows are read
+                    // below by other threads
   umma::fence_after_sync();
   const uint32_t tmem = *tmem_s;
   uint32_t ph = 0u;
   bool ok = true;
-  // every child row the walk reads above level 1, into L2 ahead of the dependent levels
-  // (K and V, two 128-byte lines each)
-  for (int l = 2; l <= t_new; ++l) {
-    const int64_t c0 = lv_j0[l] * a.b, c1 = min(lv_j1[l] * a.b, lv_np[l]);
-    const int64_t base = (a.row_off[l - 1] + bhi * a.slots[l - 1]) * kD;
-    for (int64_t e = tid; e < (c1 - c0) * 4; e += kExtendThreads)
-      prefetch_l2(((e & 2) ? a.v_node : a.k_node) + base + (c0 + (e >> 2)) * kD + (e & 1) * (kD / 2));
-  }
+  Head hs = head_start(1);  // level 1's (the token rows before the new one)
 
   for (int l = 1; l <= t_new && ok; ++l) {
     const int64_t span_prev = a.span[l - 1];
     const int64_t n_prev = lv_np[l], j0 = lv_j0[l], j1 = lv_j1[l];
-    const uint16_t *src = l == 1 ? (is_v ? a.v_tok : a.k_tok) + tok_base
-                                 : (is_v ? a.v_node : a.k_node) + (a.row_off[l - 1] + bhi * a.slots[l - 1]) * kD;
+    const uint16_t *src = level_rows(l - 1);
     uint16_t *dk = a.k_node + (a.row_off[l] + bhi * a.slots[l]) * kD;
     uint16_t *dv = a.v_node + (a.row_off[l] + bhi * a.slots[l]) * kD;
+    // one node whose last child the thread holds: the head start plus that child
+    const bool single = have_carry && j1 - j0 == 1;
     for (int64_t g0 = j0; g0 < j1 && ok; g0 += umma::kM) {  // up to 128 nodes a product
       const int64_t g1 = min(j1, g0 + (int64_t)umma::kM);
-      for (int64_t j = g0; j < g1; ++j) {
-        const int64_t c0 = j * a.b, c1 = min(c0 + (int64_t)a.b, n_prev);
-        // the level below's row of child c (tokens through the page table when paged)
-        auto child = [&](int64_t c) -> int64_t { return l == 1 ? tok_row(c) : c; };
-        float sum = 0.f;
-#pragma unroll 16
-        for (int64_t c = c0; c < c1; ++c) {
-          const int64_t r = child(c);
-          if (r >= 0) sum += bf16_lo(src[r * kD + d]);
+      const int cnt = (int)(g1 - g0);
+      // the key mean's three bf16 parts into row m of the means' operand
+      auto put_key_mean = [&](int m, float mean) {
+        uint32_t p0, p1, p2;
+        umma::split3(mean, p0, p1, p2);
+        const int off = umma::operand_offset(m, d);
+        *reinterpret_cast<uint16_t *>(Mop + off) = (uint16_t)p0;
+        *reinterpret_cast<uint16_t *>(Mop + umma::kPartBytes + off) = (uint16_t)p1;
+        *reinterpret_cast<uint16_t *>(Mop + 2 * umma::kPartBytes + off) = (uint16_t)p2;
+      };
+      if (!dims) {
+      } else if (single) {
+        float sum = hs.pre + carry;
+        if (is_v) {
+          if (hs.part) sum = __fmaf_rn(hs.f1, carry, sum);
+          const uint32_t vbits = f32_to_bf16_bits(sum / hs.wsum);
+          *hs.v_dst = (uint16_t)vbits;
+          carry = bf16_lo(vbits);  // the value as stored: the next level's last child
+        } else {
+          put_key_mean(0, sum / hs.nch);
         }
-        const float nch = (float)(c1 - c0);
-        if (is_v) {  // token-weighted: the level's last child gets its share tokens / span_prev
-          float wsum = nch;
-          if (c1 == n_prev && c1 > c0) {
-            const int64_t last_tokens = length - (c1 - 1) * span_prev;
-            if (last_tokens < span_prev) {
-              const float f1 = (float)last_tokens / (float)span_prev - 1.f;
-              const int64_t r = child(c1 - 1);
-              sum = __fmaf_rn(f1, r >= 0 ? bf16_lo(src[r * kD + d]) : 0.f, sum);
-              wsum += f1;
+      } else {
+        for (int64_t j = g0; j < g1; ++j) {
+          const int64_t c0 = j * a.b, c1 = min(c0 + (int64_t)a.b, n_prev);
+          float sum = child_sum(l, c0, c1);
+          const float nch = (float)(c1 - c0);
+          if (is_v) {  // token-weighted: the level's last child gets its share tokens / span_prev
+            float wsum = nch;
+            if (c1 == n_prev && c1 > c0) {
+              const int64_t last_tokens = length - (c1 - 1) * span_prev;
+              if (last_tokens < span_prev) {
+                const float f1 = (float)last_tokens / (float)span_prev - 1.f;
+                const int64_t r = l == 1 ? tok_row(c1 - 1) : c1 - 1;
+                sum = __fmaf_rn(f1, r >= 0 ? bf16_lo(src[r * kD + d]) : 0.f, sum);
+                wsum += f1;
+              }
             }
+            const uint32_t vbits = f32_to_bf16_bits(sum / wsum);
+            dv[j * kD + d] = (uint16_t)vbits;
+            carry = bf16_lo(vbits);
+          } else {
+            put_key_mean((int)(j - g0), sum / nch);
           }
-          dv[j * kD + d] = (uint16_t)f32_to_bf16_bits(sum / wsum);
-        } else {  // the key mean's three bf16 parts into row j - g0 of A
-          uint32_t p0, p1, p2;
-          umma::split3(sum / nch, p0, p1, p2);
-          const int off = umma::operand_offset((int)(j - g0), d);
-          *reinterpret_cast<uint16_t *>(A + off) = (uint16_t)p0;
-          *reinterpret_cast<uint16_t *>(A + umma::kPartBytes + off) = (uint16_t)p1;
-          *reinterpret_cast<uint16_t *>(A + 2 * umma::kPartBytes + off) = (uint16_t)p2;
         }
       }
       umma::fence_async_smem();
       umma::fence_before_sync();
       __syncthreads();  // the key means in place
-      if (tid == 0) {
+      if (tid == kExtendIssuer) {
         umma::fence_after_sync();
-        umma::issue_pooler(tmem, smem_u32(A), smem_u32(Bop));
+        umma::issue_pooler_t(tmem, smem_u32(Wop), smem_u32(Mop), (cnt + 15) & ~15);
         umma::commit(bar);
       }
+      // the next level's head start while the tensor cores work (with one node rebuilt here,
+      // its children before the last are rows this launch does not change)
+      if (j1 - j0 == 1) hs = head_start(l + 1);
       const bool done = __all_sync(0xffffffffu, mbar_wait(bar, ph));  // one answer a warp
       ph ^= 1u;
       umma::fence_after_sync();
-      if (done) {  // keys of nodes g0 .. g1-1: warp w reads lanes 32 (w % 4) .., columns 64 (w / 4) ..
-        const int rq = warp & 3, ch = warp >> 2, row = 32 * rq + lane;
-        uint32_t v0[32], v1[32];
-        const uint32_t t0 = tmem + ((uint32_t)(32 * rq) << 16) + 64u * ch;
-        umma::tmem_ld32(t0, v0);
-        umma::tmem_ld32(t0 + 32, v1);
-        umma::tmem_wait_ld();
-        if (row < g1 - g0) {
-          uint4 *dst = reinterpret_cast<uint4 *>(dk + (g0 + row) * kD + 64 * ch);
+      if (done && warp < 4) {
+        // keys of nodes g0 .. g1-1: key thread d reads accumulator lane d (warp w, lanes
+        // 32w ..), one column a node; a warp stores 64 contiguous bytes of each row
+        uint32_t v[32];
+        if (cnt == 1) {  // one node: column 0, kept as the next level's last child
+          umma::tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16), v);
+          umma::tmem_wait_ld();
+          const uint32_t kbits = f32_to_bf16_bits(__uint_as_float(v[0]));
+          dk[g0 * kD + d] = (uint16_t)kbits;
+          carry = bf16_lo(kbits);
+        } else {
+          for (int cb = 0; cb < cnt; cb += 32) {
+            umma::tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)cb, v);
+            umma::tmem_wait_ld();
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            dst[q] = make_uint4(pack_bf16x2(__uint_as_float(v0[8 * q]), __uint_as_float(v0[8 * q + 1])),
-                                pack_bf16x2(__uint_as_float(v0[8 * q + 2]), __uint_as_float(v0[8 * q + 3])),
-                                pack_bf16x2(__uint_as_float(v0[8 * q + 4]), __uint_as_float(v0[8 * q + 5])),
-                                pack_bf16x2(__uint_as_float(v0[8 * q + 6]), __uint_as_float(v0[8 * q + 7])));
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            dst[4 + q] = make_uint4(pack_bf16x2(__uint_as_float(v1[8 * q]), __uint_as_float(v1[8 * q + 1])),
-                                    pack_bf16x2(__uint_as_float(v1[8 * q + 2]), __uint_as_float(v1[8 * q + 3])),
-                                    pack_bf16x2(__uint_as_float(v1[8 * q + 4]), __uint_as_float(v1[8 * q + 5])),
-                                    pack_bf16x2(__uint_as_float(v1[8 * q + 6]), __uint_as_float(v1[8 * q + 7])));
+            for (int i = 0; i < 32; ++i)
+              if (cb + i < cnt) dk[(g0 + cb + i) * kD + d] = (uint16_t)f32_to_bf16_bits(__uint_as_float(v[i]));
+          }
         }
       }
+      // the accumulator is read and these rows are written before the next product is
+      // issued and the next level reads them (the product has read the means' operand)
+      umma::fence_before_sync();
       if (!__syncthreads_and(done)) {
         // the product did not complete within the wait limit: report it; the walk stops
-        if (tid == 0) {
+        if (tid == kExtendIssuer) {
           if (a.err) atomicOr(a.err, kErrTimeout);
           atomicOr(&g_build_err, kErrTimeout);
           mbar_wait(bar, ph ^ 1u);  // a last bounded wait before the accumulator is freed
         }
         ok = false;
       }
-      umma::fence_before_sync();
-      __syncthreads();  // A is rewritten next, and the next level reads these rows
     }
+    have_carry = j1 - j0 == 1;  // the node rebuilt here is the next level's last child
   }
   umma::fence_before_sync();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == kExtendIssuer / 32) {
     umma::fence_after_sync();
     umma::tmem_dealloc(tmem, umma::kTmemCols);
   }

@@ -1,7 +1,12 @@
 // Pooler product on the 5th-generation tensor cores (tcgen05, accumulator in TMEM).
 //
 // key = W @ mean for up to 128 nodes at once: D[m][o] = sum_k A[m][k] * B[o][k] with
-// A = the nodes' fp32 key means and B = W (row-major [o][k], i.e. K-major).  A single
+// A = the nodes' fp32 key means and B = W (row-major [o][k], i.e. K-major), or with the
+// roles exchanged (A = W, B = the means, D[o][m]) where few nodes need a product: an MMA
+// instruction costs about the same at N = 16 as at N = 128, 2.5K against 3.3K cycles for the
+// 48 of a product, so a short N helps only a little, and both forms give each element
+// the same fp32 result (checked element by element on B200, and by the append-equals-build
+// tests).  A single
 // bf16 pass would round the operands to 8 bits, well above the precision of a stored bf16
 // row, so each fp32 operand is split exactly into three bf16 parts x = x0 + x1 + x2
 // (x0 = bf16(x), x1 = bf16(x - x0), x2 = bf16(x - x0 - x1)) and the six products whose
@@ -40,8 +45,12 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr) {
   return (uint64_t)((saddr >> 4) & 0x3fffu) | ((uint64_t)(kLBO >> 4) << 16) | ((uint64_t)(kSBO >> 4) << 32) |
          (1ull << 46);
 }
-// Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, both K-major, N = 128, M = 128.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kN >> 3) << 17) | ((uint32_t)(kM >> 4) << 24);
+// Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, both K-major, M = 128,
+// N = n (a multiple of 16 up to 256).
+__host__ __device__ constexpr uint32_t idesc_n(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kM >> 4) << 24);
+}
+constexpr uint32_t kIdesc = idesc_n(kN);
 
 // the six products (A part, B part), smallest terms first
 __host__ __device__ constexpr int prod_a(int i) { return i == 0 ? 1 : i == 1 ? 2 : i == 2 ? 0 : i == 3 ? 1 : i == 4 ? 0 : 0; }
@@ -83,11 +92,12 @@ __device__ __forceinline__ void fence_after_sync() { asm volatile("tcgen05.fence
 // generic-proxy writes to shared memory become visible to the tensor cores' reads
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-__device__ __forceinline__ void mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+__device__ __forceinline__ void mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                    uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\ttcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(
           tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 // arrives on the mbarrier once every MMA issued before it by this thread has completed
@@ -105,7 +115,24 @@ __device__ __forceinline__ void issue_pooler(uint32_t tmem_d, uint32_t a_s, uint
     const uint32_t a0 = a_s + prod_a(pi) * kPartBytes, b0 = b_s + prod_b(pi) * kPartBytes;
 #pragma unroll
     for (int ks = 0; ks < kD / 16; ++ks) {  // 16 k per instruction: two core matrices along K
-      mma(tmem_d, smem_desc(a0 + ks * 256), smem_desc(b0 + ks * 256), acc);
+      mma(tmem_d, smem_desc(a0 + ks * 256), smem_desc(b0 + ks * 256), kIdesc, acc);
+      acc = 1;
+    }
+  }
+}
+
+// One thread: the same six products in the same order with the operands' roles exchanged,
+// D[o][m] = sum_k W[o][k] * mean[m][k] for nodes m < n (n a multiple of 16): W's parts at
+// w_s (rows o), the means' parts at m_s (rows m).
+__device__ __forceinline__ void issue_pooler_t(uint32_t tmem_d, uint32_t w_s, uint32_t m_s, int n) {
+  const uint32_t idesc = idesc_n(n);
+  uint32_t acc = 0;
+#pragma unroll
+  for (int pi = 0; pi < kProducts; ++pi) {
+    const uint32_t w0 = w_s + prod_b(pi) * kPartBytes, m0 = m_s + prod_a(pi) * kPartBytes;
+#pragma unroll
+    for (int ks = 0; ks < kD / 16; ++ks) {
+      mma(tmem_d, smem_desc(w0 + ks * 256), smem_desc(m0 + ks * 256), idesc, acc);
       acc = 1;
     }
   }
@@ -126,14 +153,30 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// W into the B operand (three parts): element (o, k) = W[o][k].
-template <int NT>
+// W into an operand (three parts): element (o, k) = W[o][k].  A warp's 32 pieces of 4 k
+// cover rows 8g .. 8g+7 and k 16c .. 16c+15: two whole core matrices, so each 8-byte store
+// fills 256 contiguous bytes without a bank conflict (a row's pieces are 128 bytes apart).
+template <int NT, int kMaxBatch = 4>
 __device__ __forceinline__ void load_pooler_operand(const float *__restrict__ W, unsigned char *b_ops, int tid) {
-  for (int e = tid; e < kD * kD / 4; e += NT) {  // 4 consecutive k of row o
-    const float4 w = __ldg(reinterpret_cast<const float4 *>(W) + e);
-    const int o = e / (kD / 4), k = (e % (kD / 4)) * 4;
-    const float x[4] = {w.x, w.y, w.z, w.w};
-    store_row4_parts(b_ops, o, k, x);
+  constexpr int kPer = kD * kD / 4 / NT;  // pieces a thread
+  constexpr int kBatch = kPer < kMaxBatch ? kPer : kMaxBatch;  // loads in flight at once
+  static_assert(kPer * NT == kD * kD / 4 && kPer % kBatch == 0, "the thread count divides the pooler's pieces");
+#pragma unroll 1
+  for (int i0 = 0; i0 < kPer; i0 += kBatch) {
+    float4 w[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int e = tid + (i0 + i) * NT, c = e >> 5, lane = e & 31;
+      const int o = (c & 15) * 8 + (lane & 7), k = (c >> 4) * 16 + (lane >> 3) * 4;
+      w[i] = __ldg(reinterpret_cast<const float4 *>(W + o * kD + k));
+    }
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int e = tid + (i0 + i) * NT, c = e >> 5, lane = e & 31;
+      const int o = (c & 15) * 8 + (lane & 7), k = (c >> 4) * 16 + (lane >> 3) * 4;
+      const float x[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+      store_row4_parts(b_ops, o, k, x);
+    }
   }
 }
 

@@ -1,4 +1,4 @@
-// Runs the append kernel (extend_kernel: one CTA of 256 threads per (sequence, KV head)) or, with
+// Runs the append kernel (extend_kernel: one CTA of 288 threads per (sequence, KV head)) or, with
 // "mode 1", every level of the tree build (build_level_mma_kernel, one launch per level, a grid of
 // at most "grid" CTAs of 512 threads striding over tiles of 128 nodes) on host threads, one
 // std::thread per CUDA thread, over inputs read from a case directory, and writes the caches and

@@ -53,8 +53,9 @@ def extract_umma(src_path: str, out_path: str) -> None:
         if k != 1:
             raise ValueError(f"helper not found in the tcgen05 header: {fn}")
     text, k = re.subn(r"__device__ __forceinline__ void mma\(uint32_t tmem_d, .*?\n\}",
-                      "inline void mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {\n"
-                      "  mma_host(tmem_d, adesc, bdesc, kIdesc, accumulate);\n}", text, count=1, flags=re.S)
+                      "inline void mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,\n"
+                      "                uint32_t accumulate) {\n"
+                      "  mma_host(tmem_d, adesc, bdesc, idesc, accumulate);\n}", text, count=1, flags=re.S)
     if k != 1:
         raise ValueError("mma not found in the tcgen05 header")
     text, k = re.subn(r"__device__ __forceinline__ void commit\(uint64_t \*bar\) \{.*?\n\}",

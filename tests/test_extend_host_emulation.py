@@ -156,6 +156,8 @@ def _run(emu_bin, tmp_path, lens, hkv, C, b, P=None, per_seq=False, seed=1):
     ([1023], 1, 1, 4),           # 1024 = 4^5: a new top level appears
     ([700, 700], 1, 40, 16),     # several level-1 nodes in one walk
     ([0], 2, 9, 4),              # an empty cache: one level of 3 nodes built from scratch
+    ([4096], 1, 1, 16),          # one token: levels 1-2 on the single-node path, level 3 new (2 nodes)
+    ([4111], 1, 1, 16),          # one token completing a level-1 node (its 16th child)
 ])
 def test_append_matches_oracle(emu_bin, tmp_path, lens, hkv, C, b):
     _run(emu_bin, tmp_path, lens, hkv, C, b)
@@ -165,9 +167,13 @@ def test_append_with_per_sequence_lengths(emu_bin, tmp_path):
     _run(emu_bin, tmp_path, [700, 1022, 0, 64], 1, 3, 4, per_seq=True, seed=4)
 
 
-@pytest.mark.parametrize("P", [1, 16])
-def test_append_into_a_paged_cache(emu_bin, tmp_path, P):
-    _run(emu_bin, tmp_path, [600, 301], 1, 5, 4, P=P, per_seq=True, seed=P)
+def test_append_one_token_with_per_sequence_lengths(emu_bin, tmp_path):
+    _run(emu_bin, tmp_path, [700, 1023, 0, 4, 65], 1, 1, 4, per_seq=True, seed=6)
+
+
+@pytest.mark.parametrize("P,C", [(1, 5), (16, 5), (16, 1)])
+def test_append_into_a_paged_cache(emu_bin, tmp_path, P, C):
+    _run(emu_bin, tmp_path, [600, 301], 1, C, 4, P=P, per_seq=True, seed=P + C)
 
 
 def _run_build(emu_bin, tmp_path, lens, hkv, b, grid, P=None, per_seq=False, seed=3):
