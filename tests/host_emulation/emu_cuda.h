@@ -230,6 +230,7 @@ struct MBar {
   long completed = 0;  // phases completed so far
 };
 MBar &mbar_of(const void *p);
+inline bool g_mbar_stuck = false;  // every mbarrier wait fails (the timeout path)
 inline void mbar_complete_if_done(MBar &b) {
   if (b.pending == 0 && b.tx == 0) {
     ++b.completed;

@@ -28,7 +28,8 @@ inline uint32_t order_key(float f) {
 inline uint32_t smem_u32(const void *p) {
   return (uint32_t)(static_cast<const unsigned char *>(p) - emu::t_smem);
 }
-constexpr uint32_t kMbarPolls = 1u << 16;
+// the poll limit of a bounded wait; the "stuck" case lowers it (every wait then runs out)
+inline uint32_t kMbarPolls = 1u << 16;
 inline void mbar_init(uint64_t *bar, uint32_t count) {
   emu::MBar &b = emu::mbar_of(bar);
   std::lock_guard<std::mutex> lk(b.mu);
@@ -44,6 +45,10 @@ inline void mbar_arrive(uint64_t *bar) {
   emu::mbar_complete_if_done(b);
 }
 inline bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  if (emu::g_mbar_stuck) {  // a barrier that never completes: the wait must give up
+    std::this_thread::yield();
+    return false;
+  }
   emu::MBar &b = emu::mbar_of(bar);
   bool done;
   {

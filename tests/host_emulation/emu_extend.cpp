@@ -170,6 +170,12 @@ int main(int argc, char **argv) {
     a.span[l] = lists["span"].at(l);
   }
   const int blocks = (int)kv["batch"] * a.hkv;
+  uint32_t err_word = 0;
+  a.err = &err_word;
+  if ((int)kv["stuck"] == 1) {  // no product ever completes: the kernels must report and return
+    emu::g_mbar_stuck = true;
+    recsa::kMbarPolls = 64;
+  }
   if ((int)kv["mode"] == 1) {  // the whole build, level by level, over `length` tokens
     const int64_t length = (int64_t)kv["length"];
     const int grid_cap = (int)kv["grid"];
@@ -216,6 +222,7 @@ int main(int argc, char **argv) {
         run_block([&] { extend_kernel<false>(a); }, kExtendSmem, blk, blocks, kExtendThreads);
     }
   }
+  std::ofstream(dir + "/err.txt") << err_word << " " << recsa::g_build_err << "\n";
   write_bin(dir + "/k_tok_out.bin", ktok);
   write_bin(dir + "/v_tok_out.bin", vtok);
   write_bin(dir + "/k_node_out.bin", knode);

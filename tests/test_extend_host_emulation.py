@@ -9,7 +9,9 @@ slots must hold the new rows bit for bit and every node row must meet the node-r
 bar against the oracle's tree over the longer cache — for equal lengths, per-sequence
 lengths and a paged token cache.  The level-build kernel runs the same way over every level
 (a grid that strides over the level's nodes, or a node per warp), its node rows held to the
-oracle's trees, with per-sequence lengths and a paged cache too.
+oracle's trees, with per-sequence lengths and a paged cache too.  Both kernels also run with
+a tensor-core product that never completes, to check that their bounded waits report the
+timeout and return.
 """
 
 import math
@@ -53,10 +55,19 @@ def _tree_rows(t, lv):
     return O.f64_to_bf16_bits(t.keys[lv]), O.f64_to_bf16_bits(t.values[lv])
 
 
-def _run(emu_bin, tmp_path, lens, hkv, C, b, P=None, per_seq=False, seed=1):
+TIMEOUT_BIT = 4  # kErrTimeout, the device error word's bit for a bounded wait that ran out
+
+
+def _timeout_words(d):
+    """The emulated call's error words: the call's own (append) and the build kernels'."""
+    return [int(x) for x in open(d / "err.txt").read().split()]
+
+
+def _run(emu_bin, tmp_path, lens, hkv, C, b, P=None, per_seq=False, seed=1, stuck=False):
     """Oracle trees over `lens`, the kernel appends C tokens per sequence, check against the
     oracle's trees over lens + C.  per_seq: the kernel reads the lengths from seq_len (else
-    every sequence has max(lens) and lens must be equal)."""
+    every sequence has max(lens) and lens must be equal).  stuck: no tensor-core product ever
+    completes; the kernel must report the timeout and return (returns the error words)."""
     B = len(lens)
     L = max(lens)
     cap = L + C
@@ -93,7 +104,7 @@ def _run(emu_bin, tmp_path, lens, hkv, C, b, P=None, per_seq=False, seed=1):
 
     span = [min(b ** lv, 1 << 62) for lv in range(R.MAX_LEVELS + 1)]
     prm = dict(batch=B, hkv=hkv, b=b, capacity=cap, at=L, chunk=C,
-               levels=len(O.level_counts(L + C, b)) - 1, page_shift=0, num_pages=0)
+               levels=len(O.level_counts(L + C, b)) - 1, page_shift=0, num_pages=0, stuck=int(stuck))
     pages = None
     k_in, v_in = kb, vb
     if P:
@@ -109,7 +120,7 @@ def _run(emu_bin, tmp_path, lens, hkv, C, b, P=None, per_seq=False, seed=1):
             for j in range(pps):
                 k_in[pages[s, j]] = kb[s, :, j * P:(j + 1) * P]
                 v_in[pages[s, j]] = vb[s, :, j * P:(j + 1) * P]
-    d = tmp_path / f"case_{B}_{hkv}_{L}_{C}_{b}_{P}_{int(per_seq)}"
+    d = tmp_path / f"case_{B}_{hkv}_{L}_{C}_{b}_{P}_{int(per_seq)}_{int(stuck)}"
     d.mkdir()
     with open(d / "params.txt", "w") as f:
         for key, val in prm.items():
@@ -127,6 +138,8 @@ def _run(emu_bin, tmp_path, lens, hkv, C, b, P=None, per_seq=False, seed=1):
     np.ascontiguousarray(inp["pooler"].numpy(), dtype=np.float32).tofile(d / "pooler.bin")
     r = subprocess.run([emu_bin, str(d)], capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, (r.stdout[-2000:], r.stderr[-4000:])
+    if stuck:
+        return _timeout_words(d)
 
     k_out = np.fromfile(d / "k_tok_out.bin", np.uint16).reshape(k_in.shape)
     v_out = np.fromfile(d / "v_tok_out.bin", np.uint16).reshape(v_in.shape)
@@ -176,7 +189,7 @@ def test_append_into_a_paged_cache(emu_bin, tmp_path, P, C):
     _run(emu_bin, tmp_path, [600, 301], 1, C, 4, P=P, per_seq=True, seed=P + C)
 
 
-def _run_build(emu_bin, tmp_path, lens, hkv, b, grid, P=None, per_seq=False, seed=3):
+def _run_build(emu_bin, tmp_path, lens, hkv, b, grid, P=None, per_seq=False, seed=3, stuck=False):
     """The level-build kernel over every level (at most `grid` CTAs striding over the tiles of
     128 nodes) on the CPU; each sequence's node rows against the oracle's tree over its tokens."""
     B, L = len(lens), max(lens)
@@ -188,7 +201,7 @@ def _run_build(emu_bin, tmp_path, lens, hkv, b, grid, P=None, per_seq=False, see
     node_rows, levels_cap, offs = R.tree_layout(p, B, cap)
     slots = [cap] + [math.ceil(cap / b ** lv) for lv in range(1, levels_cap + 1)]
     prm = dict(mode=1, length=L, grid=grid, batch=B, hkv=hkv, b=b, capacity=cap, at=0, chunk=0,
-               levels=len(O.level_counts(L, b)) - 1, page_shift=0, num_pages=0)
+               levels=len(O.level_counts(L, b)) - 1, page_shift=0, num_pages=0, stuck=int(stuck))
     k_in, v_in, pages = kb, vb, None
     if P:
         pps = cap // P
@@ -202,7 +215,7 @@ def _run_build(emu_bin, tmp_path, lens, hkv, b, grid, P=None, per_seq=False, see
             for j in range(pps):
                 k_in[pages[s, j]] = kb[s, :, j * P:(j + 1) * P]
                 v_in[pages[s, j]] = vb[s, :, j * P:(j + 1) * P]
-    d = tmp_path / f"build_{B}_{hkv}_{L}_{b}_{grid}_{P}_{int(per_seq)}"
+    d = tmp_path / f"build_{B}_{hkv}_{L}_{b}_{grid}_{P}_{int(per_seq)}_{int(stuck)}"
     d.mkdir()
     span = [min(b ** lv, 1 << 62) for lv in range(R.MAX_LEVELS + 1)]
     with open(d / "params.txt", "w") as f:
@@ -222,6 +235,8 @@ def _run_build(emu_bin, tmp_path, lens, hkv, b, grid, P=None, per_seq=False, see
     np.ascontiguousarray(inp["pooler"].numpy(), dtype=np.float32).tofile(d / "pooler.bin")
     r = subprocess.run([emu_bin, str(d)], capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, (r.stdout[-2000:], r.stderr[-4000:])
+    if stuck:
+        return _timeout_words(d)
     kn_out = np.fromfile(d / "k_node_out.bin", np.uint16).reshape(zeros.shape)
     vn_out = np.fromfile(d / "v_node_out.bin", np.uint16).reshape(zeros.shape)
     mism = total = 0
@@ -247,3 +262,19 @@ def test_level_build_matches_oracle(emu_bin, tmp_path, grid):
 
 def test_level_build_with_per_sequence_lengths_and_pages(emu_bin, tmp_path):
     _run_build(emu_bin, tmp_path, [700, 0, 301, 64], 1, 4, 3, P=8, per_seq=True)
+
+
+# The timeout path: a tensor-core product that never completes (on the host, every mbarrier
+# wait gives up).  The kernels must set the timeout bit, stop, and return: the emulator's
+# rendezvous would report a thread left waiting, and AddressSanitizer a bad access.
+@pytest.mark.parametrize("C", [1, 5])  # the single-token path and the general one
+def test_append_reports_a_product_that_never_completes(emu_bin, tmp_path, C):
+    call_word, build_word = _run(emu_bin, tmp_path, [1000], 2, C, 4, stuck=True)
+    assert call_word & TIMEOUT_BIT and build_word & TIMEOUT_BIT
+
+
+@pytest.mark.parametrize("grid", [1, 1000])  # the wait inside the tile loop, and the last one
+def test_level_build_reports_a_product_that_never_completes(emu_bin, tmp_path, grid):
+    _, build_word = _run_build(emu_bin, tmp_path, [1000, 1000], 2, 4, grid, stuck=True)
+    assert build_word & TIMEOUT_BIT
+
