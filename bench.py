@@ -5,8 +5,9 @@ heads, head_dim 128, b = 16, k = 8, one query per sequence), each step one
 recsa_decode call over a tree built beforehand, L2 flushed between steps.  The same
 line carries the roofline of the attend kernel, an end-to-end figure through host
 buffers, a sweep of independent queries per sequence, causal prefill tokens/s
-(524K + 8K chunk, and 1M + 8K), the 2M-token tree build in GB/s, 2M decode latency
-and the fp64 oracle timed on the host cores.
+(524K + 8K chunk, and 1M + 8K), the 2M-token tree build in GB/s, 2M decode latency,
+decode at 131K (B = 8), the decode loop (append + decode), per-sequence lengths, a paged
+cache, and the fp64 oracle timed on the host cores.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--quick]
 
@@ -517,6 +518,29 @@ def leg_decode_paged(R, timer, args, dist_on):
     return res
 
 
+def leg_decode_131k(R, timer, args, dist_on, hbm_peak):
+    """Decode at 131K tokens, B = 8 (one query per sequence, per-(KV head, channel) scales on
+    K and V): queries/s and the logical bytes against the HBM roofline."""
+    w = I.WORKLOADS["decode_131k"]
+    inp = I.decode_inputs(w, device="cuda")
+    p = R.params(num_kv_heads=w.kv_heads, num_q_heads=w.q_heads, branching=w.branching, top_k=w.top_k)
+    tree, ws = make_tree(R, p, inp, w.length)
+    q = inp["q"]
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
+    rows = decode_entries(R, p, tree, ws, q)
+    nb = rows * ROW + q.numel() * 2 + out.numel() * 2
+    steps = max(20, args.steps // 10) if not args.quick else 20
+    per, _ = timer.run(lambda: R.decode(p, tree, q, out, ws), steps, 3)
+    t = max_over_ranks(sum(per), dist_on) / steps
+    R.check_device_errors(ws)
+    del tree, ws, inp
+    torch.cuda.empty_cache()
+    return {"workload": f"decode_131k: B={w.batch}, L={w.length}, Hq={w.q_heads}, Hkv={w.kv_heads}, "
+                        f"b={w.branching}, k={w.top_k}, 1 query per sequence",
+            "queries_per_s": w.batch / t, "us_per_call": t * 1e6, "rows_read_per_call": rows,
+            "logical_GBps": nb / t / 1e9, "frac": nb / t / 1e9 / hbm_peak}
+
+
 def leg_build_2m(R, timer, args, dist_on, hbm_peak):
     w = I.WORKLOADS["build_decode_2m"]
     inp = I.decode_inputs(w, device="cuda")
@@ -862,6 +886,7 @@ def run_gpu(args):
         extra["prefill"] = leg_prefill(R, timer, args, dist_on, hbm_peak, "prefill_524k", 524288)
         extra["prefill_1m"] = leg_prefill(R, timer, args, dist_on, hbm_peak, "prefill_1m", 1 << 20)
         extra["build_2m"] = leg_build_2m(R, timer, args, dist_on, hbm_peak)
+        extra["decode_131k"] = leg_decode_131k(R, timer, args, dist_on, hbm_peak)
         extra["decode_loop_1m"] = leg_decode_loop(R, timer, args, dist_on)
         extra["decode_varlen"] = leg_decode_varlen(R, timer, args, dist_on)
         extra["decode_paged_1m"] = leg_decode_paged(R, timer, args, dist_on)
