@@ -173,7 +173,7 @@ recsa_status check_debug(const recsa_params *p, const recsa_debug *d) {
     return fail(RECSA_ERR_INVALID_ARGUMENT, "sel_idx needs 1 <= top_k <= %d and sel_levels >= 1", kDebugMaxK);
   if (d->cluster_size != 0 && d->cluster_size != 1 && d->cluster_size != 2 && d->cluster_size != 4)
     return fail(RECSA_ERR_INVALID_ARGUMENT, "cluster_size %d (0, 1, 2 or 4)", d->cluster_size);
-  if (d->kernel < 0 || d->kernel > 3) return fail(RECSA_ERR_INVALID_ARGUMENT, "kernel %d (0 .. 3)", d->kernel);
+  if (d->kernel < 0 || d->kernel > 4) return fail(RECSA_ERR_INVALID_ARGUMENT, "kernel %d (0 .. 4)", d->kernel);
   return RECSA_OK;
 }
 

@@ -573,11 +573,16 @@ __device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
-template <int G, int CS, bool kPaged = false>
-__global__ void __launch_bounds__(kCtaThreads, 1) attend_cta_kernel(const AttendArgs a) {
-  constexpr int RPH = (CS == 4 || G == 8) ? 2 : 4;  // rows per half-warp per pass (register budget)
-  constexpr int PASS = kHalfWarps * RPH;              // rows per CTA per pass
-  constexpr bool PIPE = RPH == 2;                      // gather the next level before folding this one
+// kTwoPerSm: the instance for more tiles than SMs (one CTA a tile): two CTAs share an SM
+// (128 registers a thread), with fewer rows in flight and no gather of the next level ahead;
+// a tile takes longer (1M, one wave: 66 against 52 us) but two run at once (512 tiles: 141
+// against 179 us).
+template <int G, int CS, bool kPaged = false, bool kTwoPerSm = false>
+__global__ void __launch_bounds__(kCtaThreads, kTwoPerSm ? 2 : 1) attend_cta_kernel(const AttendArgs a) {
+  static_assert(!kTwoPerSm || CS == 1, "two CTAs per SM only for a CTA per tile");
+  constexpr int RPH = (CS == 4 || G == 8 || kTwoPerSm) ? 2 : 4;  // rows per half-warp per pass (register budget)
+  constexpr int PASS = kHalfWarps * RPH;                           // rows per CTA per pass
+  constexpr bool PIPE = RPH == 2 && !kTwoPerSm;  // gather the next level before folding this one
   extern __shared__ __align__(128) unsigned char smem[];
   const CtaLayout Ls = cta_layout(G, CS, a.max_cand, a.own_max, a.top_k);
   int *misc = reinterpret_cast<int *>(smem + Ls.misc);  // see kMiscInts
@@ -1852,7 +1857,7 @@ int sm_count_cached() {
 }
 
 template <int G, int CS, bool kPaged>
-int launch_cta(const AttendArgs &args, cudaStream_t stream) {
+int launch_cta(const AttendArgs &args, cudaStream_t stream, bool two_per_sm = false) {
   AttendArgs a = args;
   a.own_max = ((a.max_cand + CS - 1) / CS + 31) / 32 * 32;
   const CtaLayout L = cta_layout(G, CS, a.max_cand, a.own_max, a.top_k);
@@ -1861,6 +1866,10 @@ int launch_cta(const AttendArgs &args, cudaStream_t stream) {
     return -1;
   }
   auto kern = attend_cta_kernel<G, CS, kPaged>;
+  // shape 4: the two-per-SM instance, where two CTAs' shared memory fits an SM (G <= 4:
+  // with 8 query heads a tile, 128 registers a thread spill)
+  if constexpr (CS == 1 && G <= 4)
+    if (two_per_sm && 2 * (L.total + 1024) <= 228 * 1024) kern = attend_cta_kernel<G, 1, kPaged, true>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
   if (e != cudaSuccess) return (int)e;
   if constexpr (CS == 1) {
@@ -1954,6 +1963,7 @@ int launch_lean(const AttendArgs &a, int CS, cudaStream_t stream) {
 template <int G, bool kPaged>
 int launch_gp(const AttendArgs &a, int kernel, int CS, cudaStream_t stream) {
   if (kernel == 2) return launch_warp<G, kPaged>(a, stream);
+  if (kernel == 4) return launch_cta<G, 1, kPaged>(a, stream, true);
   if (kernel == 3) {
     const int rc = launch_lean<G, kPaged>(a, CS, stream);
     if (rc != kNoLeanShape) return rc;
@@ -2015,10 +2025,10 @@ int launch_attend(const AttendLaunch &l, void *stream) {
   int kernel = l.kernel;
   // A cluster (or CTA) per tile while every tile has its own SM, the lean cluster kernel
   // wherever its shape applies (launch_g falls back to the CTA kernel otherwise).  Up to
-  // 4 waves of tiles a CTA per tile still finishes first: a wave costs about a fifth of
-  // what one warp takes to walk a tile alone, and the warp-per-tile grid holds every tile
-  // at once only beyond that.
-  if (kernel == 0) kernel = (a.tiles <= sms) ? 3 : (a.tiles <= 4 * sms) ? 1 : 2;
+  // 4 waves of tiles a CTA per tile, two sharing an SM, still finishes first (1M, B = 4:
+  // 256 tiles 75 us, 512 tiles 141 us, against 94 and 179 us one CTA per SM and ~245 us
+  // for the warp-per-tile grid, which holds every tile at once only beyond that).
+  if (kernel == 0) kernel = (a.tiles <= sms) ? 3 : (a.tiles <= 4 * sms) ? 4 : 2;
   int CS = l.cluster_size;
   if ((kernel == 1 || kernel == 3) && CS == 0) CS = (a.tiles * 4 <= sms) ? 4 : (a.tiles * 2 <= sms) ? 2 : 1;
   int rc;

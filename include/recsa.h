@@ -142,13 +142,15 @@ typedef struct recsa_tree {
  *   sel_idx  : int32 [tiles][sel_levels][top_k]; slot (l-1) receives the node indices
  *              kept at level l (ascending, -1 padded).  Needs top_k <= 64.
  *   entries  : int32 [tiles][2]; keys scored and values folded by the tile (rows read).
- *   kernel   : 0 = automatic (3 while tiles <= SM count, 1 up to 4 x SM count tiles,
+ *   kernel   : 0 = automatic (3 while tiles <= SM count, 4 up to 4 x SM count tiles,
  *              2 beyond); 1 = one CTA (or a cluster of cluster_size CTAs) per tile;
  *              2 = one warp per tile, the throughput shape for many tiles; 3 = one
  *              cluster of 2 or 4 CTAs per tile in which every CTA ranks all of a
  *              level's scores (one cluster and one block barrier per level), where a
- *              level's candidates fit its registers, else shape 1.  Results agree up
- *              to fp32 rounding.
+ *              level's candidates fit its registers, else shape 1; 4 = one CTA per
+ *              tile with two CTAs sharing an SM (fewer rows in flight per CTA), where
+ *              the group has at most 4 query heads and two CTAs' shared memory fits,
+ *              else shape 1 with one CTA per tile.  Results agree up to fp32 rounding.
  *   cluster_size: with kernel 1 or 3: 0 = automatic, or 1, 2, 4 CTAs per tile. */
 typedef struct recsa_debug {
   int32_t *sel_idx;

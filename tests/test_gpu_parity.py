@@ -164,6 +164,19 @@ def test_decode_odd_shapes(B, hkv, G, L, b, k, Q, kernel, cluster_size):
     _decode_and_check(case, oracle_trees(inp, b, L), inp["q"], k, cluster_size, kernel)
 
 
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("kernel", [0, 1, 4])
+def test_decode_more_tiles_than_sms(G, kernel):
+    # 40 queries per sequence: 160 to 640 tiles, more than the B200's 148 SMs, where a CTA per
+    # tile runs two CTAs per SM (G <= 4) and the automatic choice picks that shape up to 592
+    B, hkv, L, b, k, Q = 2, max(2, 8 // G), 3000, 8, 4, 40
+    inp = I.random_case(B, L, hkv, hkv * G, Q, seed=11 * G + kernel)
+    case = GpuCase(inp, _params(hkv, G, b, k), L)
+    case.build()
+    assert B * hkv * Q > 148
+    _decode_and_check(case, oracle_trees(inp, b, L), inp["q"], k, 0, kernel)
+
+
 @pytest.mark.parametrize("kernel,cluster_size", SHAPES)
 def test_decode_ties_keep_lower_index(kernel, cluster_size):
     L, b, k = 4096, 8, 3
@@ -231,7 +244,7 @@ def _prefill_check(B, hkv, G, L, C, b, k, cluster_size=0, seed=1, kernel=0):
     (1, 2, 2, 777, 260, 3, 3),     # partial nodes at every level, b = 3
     (1, 1, 8, 250, 20, 16, 8),     # the chunk crosses into a new top level
 ])
-@pytest.mark.parametrize("kernel", [0, 1, 2])
+@pytest.mark.parametrize("kernel", [0, 1, 2, 4])
 def test_prefill_chunk_matches_oracle(B, hkv, G, L, C, b, k, kernel):
     stats, _ = _prefill_check(B, hkv, G, L, C, b, k, kernel=kernel)
     print("prefill", kernel, stats)
