@@ -223,7 +223,8 @@ RECSA_API recsa_status recsa_decode_host(const recsa_params *params, const recsa
  * v_new go to token slots L .. L+count-1 (L = tree->length), and every node whose span
  * meets those slots is rebuilt from its children -- the new tokens' ancestors, O(T)
  * nodes per (sequence, head) for one token -- plus any level that becomes new.  The
- * result equals recsa_build_tree over L + count tokens.  This is the cache update of a
+ * result equals recsa_build_tree over L + count tokens bit for bit (both form a key
+ * with the same split-bf16 tensor-core product of the pooler).  This is the cache update of a
  * decode loop: append the step's token, then recsa_decode its query at the new length.
  * On success tree->length becomes L + count (host-side update; the device work is
  * still queued).
@@ -285,10 +286,13 @@ RECSA_API recsa_status recsa_decode_no_alloc(const recsa_params *params, const r
                                              int32_t num_queries, void *out, int32_t out_is_fp32,
                                              recsa_stream_t stream);
 
-/* Synchronise `stream`, then read and clear the workspace's device error word.
+/* Synchronise `stream`, then read and clear the workspace's device error word and the
+ * library's own word for the build and append kernels (which take no workspace).
  * Returns RECSA_OK, RECSA_ERR_DEVICE_CHECK (an index out of range, or a workspace
  * that was not initialised for the call), RECSA_ERR_TIMEOUT (a bounded wait ran
- * out), or RECSA_ERR_CUDA. */
+ * out: the attend kernels' none, the build and append kernels' wait on a tensor-core
+ * product of the pooler, after which those keys are left unwritten), or
+ * RECSA_ERR_CUDA. */
 RECSA_API recsa_status recsa_check_device_errors(void *ws, recsa_stream_t stream);
 
 /* Static name of a status code. */
