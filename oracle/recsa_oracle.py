@@ -137,6 +137,30 @@ class Tree:
         return len(self.keys) - 1
 
 
+def build_level(kp, vp, cp, pooler, b: int, storage: str = "bf16"):
+    """One level above [n_prev] rows kp, vp of token counts cp: node j covers children
+    j*b .. j*b+b-1 (the last node fewer), key = W @ mean(children keys) (R1), value = the
+    count-weighted mean of the children values (R3), count = the children's sum.  With
+    bf16 storage the rows are rounded as stored (R2).  Returns (keys, values, counts)."""
+    W = np.asarray(pooler, dtype=np.float64)
+    n_prev = kp.shape[0]
+    n = -(-n_prev // b)
+    kn = np.empty((n, HEAD_DIM))
+    vn = np.empty((n, HEAD_DIM))
+    cn = np.empty(n)
+    for j in range(n):
+        c0, c1 = j * b, min((j + 1) * b, n_prev)
+        mean_key = kp[c0:c1].sum(axis=0) / (c1 - c0)
+        kn[j] = W @ mean_key
+        w = cp[c0:c1]
+        vn[j] = (w[:, None] * vp[c0:c1]).sum(axis=0) / w.sum()
+        cn[j] = w.sum()
+    if storage == "bf16":
+        kn = round_to_bf16(kn)
+        vn = round_to_bf16(vn)
+    return kn, vn, cn
+
+
 def build_tree(k_tok, v_tok, pooler, b: int, storage: str = "bf16") -> Tree:
     """Build the summary tree of one (sequence, KV head).
 
@@ -147,26 +171,11 @@ def build_tree(k_tok, v_tok, pooler, b: int, storage: str = "bf16") -> Tree:
         raise ValueError(storage)
     k_tok = np.asarray(k_tok, dtype=np.float64)
     v_tok = np.asarray(v_tok, dtype=np.float64)
-    W = np.asarray(pooler, dtype=np.float64)
     L = k_tok.shape[0]
     ns = level_counts(L, b)
     keys, values, counts = [k_tok], [v_tok], [np.ones(L)]
-    for lvl in range(1, len(ns)):
-        kp, vp, cp = keys[-1], values[-1], counts[-1]
-        n_prev, n = ns[lvl - 1], ns[lvl]
-        kn = np.empty((n, HEAD_DIM))
-        vn = np.empty((n, HEAD_DIM))
-        cn = np.empty(n)
-        for j in range(n):
-            c0, c1 = j * b, min((j + 1) * b, n_prev)
-            mean_key = kp[c0:c1].sum(axis=0) / (c1 - c0)
-            kn[j] = W @ mean_key
-            w = cp[c0:c1]
-            vn[j] = (w[:, None] * vp[c0:c1]).sum(axis=0) / w.sum()
-            cn[j] = w.sum()
-        if storage == "bf16":
-            kn = round_to_bf16(kn)
-            vn = round_to_bf16(vn)
+    for _ in range(1, len(ns)):
+        kn, vn, cn = build_level(keys[-1], values[-1], counts[-1], pooler, b, storage)
         keys.append(kn)
         values.append(vn)
         counts.append(cn)

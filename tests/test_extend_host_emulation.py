@@ -171,6 +171,7 @@ def _run(emu_bin, tmp_path, lens, hkv, C, b, P=None, per_seq=False, seed=1, stuc
     ([0], 2, 9, 4),              # an empty cache: one level of 3 nodes built from scratch
     ([4096], 1, 1, 16),          # one token: levels 1-2 on the single-node path, level 3 new (2 nodes)
     ([4111], 1, 1, 16),          # one token completing a level-1 node (its 16th child)
+    ([3000], 1, 1, 2),           # b = 2: 11 levels of one node each on the single-token path
 ])
 def test_append_matches_oracle(emu_bin, tmp_path, lens, hkv, C, b):
     _run(emu_bin, tmp_path, lens, hkv, C, b)

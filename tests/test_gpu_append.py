@@ -1,7 +1,9 @@
 """GPU parity of recsa_append (token append + update of the nodes over the new tokens).
 
-The appended tree is held to the oracle's fresh build over all tokens (the node rows,
-within two bf16 ulps of each row's largest element, and the token slots bit for bit),
+The appended tree is held to the oracle level by level (each level's rows against the
+oracle's level step over the library's own rows below, within two bf16 ulps of each row's
+largest element), to the oracle's fresh build over all tokens up to 8 levels deep, the
+token slots bit for bit,
 and to the library's own full build bit for bit: both paths of the update (one launch
 walking each head's ancestor path, and the per-level launches used for long chunks)
 share the level build's per-node arithmetic.  A decode loop of append + decode is held
@@ -39,6 +41,29 @@ def _compare_nodes(case, trees):
     return mism, total
 
 
+def _compare_levels_stepwise(case, kc, vc, pooler, B, hkv, length, b):
+    """Each level's rows against the oracle's level step applied to the library's own
+    stored rows of the level below: the node-row bar for one level's arithmetic, whatever
+    the depth.  Returns (elements not bit-identical, total)."""
+    mism = total = 0
+    top = len(O.level_counts(length, b)) - 1
+    gpu = [case.node_bits(lvl) for lvl in range(1, top + 1)]
+    for s in range(B):
+        for h in range(hkv):
+            kp = O.bf16_bits_to_f64(kc[s, h, :length])
+            vp = O.bf16_bits_to_f64(vc[s, h, :length])
+            cp = np.ones(length)
+            for lvl in range(1, top + 1):
+                kn, vn, cn = O.build_level(kp, vp, cp, pooler, b)
+                gk, gv = gpu[lvl - 1][0][s, h, :kn.shape[0]], gpu[lvl - 1][1][s, h, :kn.shape[0]]
+                for got, want in ((gk, kn), (gv, vn)):
+                    m, c = check_node_rows(got, want)
+                    mism += m
+                    total += c
+                kp, vp, cp = O.bf16_bits_to_f64(gk), O.bf16_bits_to_f64(gv), cn
+    return mism, total
+
+
 def _appended_case(B, hkv, L, C, b, seed, k=2, G=4, extra=0):
     inp = I.random_case(B, L, hkv, hkv * G, 0, seed=seed, capacity=L + C + extra, chunk=C)
     case = GpuCase(inp, _params(hkv, G, b, k), L)
@@ -63,6 +88,7 @@ CASES = [
     (1, 2, 2, 30, 4),        # 8 level-1 nodes from scratch: per-level launches
     (1, 1, 100, 200, 4),     # a long chunk: per-level launches
     (3, 8, 4096, 1, 16),     # 24 (sequence, head) warps over 3 blocks
+    (1, 2, 70000, 1, 2),     # b = 2: 16 levels, one node each, carried up the single-token path
 ]
 
 
@@ -73,10 +99,17 @@ def test_append_matches_oracle(B, hkv, L, C, b):
     # token slots: the new rows in place, every other slot untouched
     assert np.array_equal(bits(case.k_tok)[:, :, :L + C], kc[:, :, :L + C])
     assert np.array_equal(bits(case.v_tok)[:, :, :L + C], vc[:, :, :L + C])
-    trees = O.build_all(kc, vc, inp["pooler"].double().numpy(), b, L + C)
-    mism, total = _compare_nodes(case, trees)
+    W = inp["pooler"].double().numpy()
+    mism, total = _compare_levels_stepwise(case, kc, vc, W, B, hkv, L + C, b)
     assert mism <= max(total, 1) * 1e-2
+    trees = O.build_all(kc, vc, W, b, L + C)
     assert case.tree.levels >= trees[0][0].top
+    # the whole tree against the oracle's own: rows rounded independently on both sides drift
+    # apart by about sqrt(depth) half-ulps as they pass up the levels, past the two-ulp bar in
+    # deep trees (b = 2, 16 levels: 2.5 ulps seen), so this holds up to 8 levels
+    if trees[0][0].top <= 8:
+        mism, total = _compare_nodes(case, trees)
+        assert mism <= max(total, 1) * 1e-2
 
 
 @pytest.mark.parametrize("B,hkv,L,C,b", CASES)
