@@ -155,6 +155,7 @@ def test_decode_k0_is_attention_over_top_summaries(kernel, cluster_size):
     (1, 1, 4, 1, 16, 8, 1),        # a single token
     (1, 2, 4, 3000, 5, 40, 1),     # many candidates per level (several gather chunks)
     (2, 1, 4, 2048, 4, 1, 4),      # k = 1
+    (1, 2, 4, 20000, 2, 2, 2),     # b = 2: 14 levels above the tokens
 ])
 @pytest.mark.parametrize("kernel,cluster_size", [(1, 1), (1, 4), (2, 0), (3, 2), (3, 4)])
 def test_decode_odd_shapes(B, hkv, G, L, b, k, Q, kernel, cluster_size):
